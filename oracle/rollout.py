@@ -1,0 +1,103 @@
+"""Chunk-wise autoregressive rollout over the sink + window cache, fp64.
+
+What it computes ([LWI] "The trick: treat video like a causal stream": the
+state is anchor tokens plus recent context, old tokens are evicted while the
+anchors are kept, each step reads the state and its result is appended;
+[WiW]: the block reads 6 anchor + 8 recent + 4 current latent frames; [RT]
+setup: 16-frame chunks = 4 latent frames, four denoising steps):
+
+  for each chunk t (frames f0 .. f0+F-1):
+      (dynamic window) evict down to the scheduled window W_t
+      for each denoising step:
+          Q_rot = RoPE3D(Q), K_rot = RoPE3D(K) at the chunk's own positions
+          O = attention(Q_rot, [K of cached frames, K_rot], [V cached, V])
+      append the last step's rotated K and V of each frame to the cache
+
+Readings: the queries of a chunk read every token of their own chunk (no
+causal mask inside a chunk); the cache stores K already rotated at its
+absolute frame index; V is not rotated; the finalized K/V are the last
+step's; with a dynamic window the eviction to W_t happens before the
+chunk's attention and appends use the largest window as capacity.
+
+Parity: pinned (equals brute-force attention over the whole concatenated
+rollout under the set-based visibility rule; a chunk's output does not change
+when later chunks change).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional
+
+import numpy as np
+
+from .attn import attention
+from .cache import CacheModel
+from .rope import rope3d, rope_positions
+
+
+@dataclasses.dataclass
+class RolloutResult:
+    outputs: List[np.ndarray]          # per (chunk, step): O of the checked rows [n, H, D]
+    lses: List[np.ndarray]             # per (chunk, step): LSE [H, n]
+    rows: List[np.ndarray]             # per (chunk, step): checked row indices
+    slot_maps: List[List[int]]         # per chunk, after its append
+    appended_slots: List[List[int]]    # per chunk: slot of each appended frame
+    evicted: List[List[int]]           # per chunk: frames evicted (dynamic evict + append)
+    visible: List[List[int]]           # per chunk: cached frames read (ascending)
+    n_keys: List[int]                  # per chunk: keys read (cached + current)
+
+
+def rollout(spec, chunks, rows_for=None, use_rope: bool = True,
+            window_schedule: Optional[List[int]] = None) -> RolloutResult:
+    """Run the rollout of ``spec`` (a RolloutSpec) over ``chunks``.
+
+    ``chunks`` yields dicts with chunk, step, frames, q, k, v as produced by
+    ``workloads.rollout_chunks``.  ``rows_for(chunk, step)`` returns the query
+    rows to evaluate (default: all).
+    """
+    T = spec.grid_h * spec.grid_w
+    scale = 1.0 / math.sqrt(spec.head_dim)
+    pairs = (spec.rope().pairs_t, spec.rope().pairs_h, spec.rope().pairs_w)
+    cap = spec.window if window_schedule is None else max(spec.window, max(window_schedule))
+    cache = CacheModel(spec.sinks, cap)
+    store: Dict[int, tuple] = {}     # frame -> (K_rot [T,H,D], V [T,H,D])
+    res = RolloutResult([], [], [], [], [], [], [], [])
+    pending_evicted: List[int] = []
+    for item in chunks:
+        c, s, frames = item["chunk"], item["step"], item["frames"]
+        q = np.asarray(item["q"], dtype=np.float64)
+        k = np.asarray(item["k"], dtype=np.float64)
+        v = np.asarray(item["v"], dtype=np.float64)
+        if s == 0 and window_schedule is not None:
+            pending_evicted = cache.evict(window_schedule[c])
+            for f in pending_evicted:
+                store.pop(f, None)
+        if use_rope:
+            t, hh, ww = rope_positions(frames, spec.grid_h, spec.grid_w)
+            q_rot = rope3d(q, t, hh, ww, pairs, spec.rope().base)
+            k_rot = rope3d(k, t, hh, ww, pairs, spec.rope().base)
+        else:
+            q_rot, k_rot = q, k
+        vis = cache.cached_frames()
+        k_all = np.concatenate([store[f][0] for f in vis] + [k_rot], axis=0)
+        v_all = np.concatenate([store[f][1] for f in vis] + [v], axis=0)
+        rows = np.arange(q.shape[0]) if rows_for is None else np.asarray(rows_for(c, s))
+        o, lse = attention(q_rot[rows], k_all, v_all, scale)
+        res.outputs.append(o)
+        res.lses.append(lse)
+        res.rows.append(rows)
+        if s == spec.steps - 1:
+            res.visible.append(vis)
+            res.n_keys.append(k_all.shape[0])
+            slots, ev = cache.append(frames)
+            for f in ev:
+                store.pop(f, None)
+            for n, f in enumerate(frames):
+                if slots[n] >= 0:
+                    store[f] = (k_rot[n * T:(n + 1) * T], v[n * T:(n + 1) * T])
+            res.appended_slots.append(slots)
+            res.evicted.append(pending_evicted + ev)
+            res.slot_maps.append(cache.slot_map())
+            pending_evicted = []
+    return res
