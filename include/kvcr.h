@@ -1,0 +1,221 @@
+/*
+ * kvcr.h -- C ABI of the sink + window chunk-attention library for B200 (sm_100a).
+ *
+ * The library implements the attention hot path of chunk-wise autoregressive
+ * video world models:
+ *
+ *   - a per-layer KV cache of pinned anchor ("sink") latent frames followed by
+ *     a sliding window of recent finalized frames, with eviction of the oldest
+ *     non-anchor frame ("LingBot-World-Infinity: The Open-Source World Model
+ *     That Refuses to Forget", sections "The trick: treat video like a causal
+ *     stream" and "How the cache keeps the world alive"; "Westlake AGI Lab's
+ *     'World in World' Steers Frozen Video Models", second paragraph: 6 anchor
+ *     + 8 recent + 4 current latent-frame slots);
+ *   - 3D (t, h, w) rotary embedding of K applied when a frame is written;
+ *   - chunk attention: the current chunk's queries attend the anchors, the
+ *     window and the chunk itself;
+ *   - attention under the MoBA training mask ("Infinite Worlds with Versatile
+ *     Interactions", causal-pretraining paragraph; "Mix Forcing: Causal
+ *     Pre-Training via Mixture Attention for Interactive World Models",
+ *     "Mix the training modes").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every call returns a kvcr_status.  On a non-OK return nothing was launched
+ *    and no state changed; kvcr_last_error() gives a message (thread-local).
+ *  - Tensors are dense, row-major, token-major: [tokens][heads][head_dim], in
+ *    the cache's dtype (bf16 or fp32).  Device pointers must be 16-byte
+ *    aligned.  Tokens of one latent frame are row-major over the (h, w) patch
+ *    grid; frames follow each other in ascending frame order.
+ *  - "stream" is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Device work is asynchronous on that stream; no call synchronises the host
+ *    except kvcr_check_status() and kvcr_trace_read().  Inputs must stay valid
+ *    until the stream has consumed them.
+ *  - Host-side bookkeeping (slot table, frame order) never reads device memory.
+ *  - The library never allocates device memory: the cache lives in one
+ *    caller-owned device buffer of kv_cache_storage_bytes() bytes.
+ *  - All compute runs in the library's own CUDA kernels; there is no CPU
+ *    fallback.
+ */
+#ifndef KVCR_H
+#define KVCR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVCR_OK = 0,
+    KVCR_EINVAL = -1,      /* null pointer, misaligned pointer, bad scalar argument */
+    KVCR_ESHAPE = -2,      /* sizes inconsistent with the cache or out of supported range */
+    KVCR_ESTATE = -3,      /* call not valid in the cache's state (frame order, no storage) */
+    KVCR_ECUDA = -4,       /* a CUDA runtime / driver call failed */
+    KVCR_ETIMEOUT = -5,    /* a kernel gave up on a bounded wait (reported by kvcr_check_status) */
+    KVCR_ESTORAGE = -6,    /* caller storage too small or misaligned */
+    KVCR_EUNSUPPORTED = -7 /* dtype / head_dim combination not built */
+} kvcr_status;
+
+typedef enum { KVCR_BF16 = 0, KVCR_F32 = 1 } kvcr_dtype;
+
+/* 3D rotary embedding of a cache.  head_dim is cut into head_dim/2 interleaved
+ * pairs (x[2i], x[2i+1]); the first pairs_t pairs rotate with the absolute
+ * latent-frame index t, the next pairs_h with the patch row h, the last pairs_w
+ * with the patch column w.  In an axis owning P pairs, pair j turns by
+ * pos * base^(-2j / (2P)).  pairs_t + pairs_h + pairs_w == head_dim / 2 and
+ * grid_h * grid_w == tokens_per_frame.  Angles are computed on the host in
+ * double precision.  The 832x464 workload uses 22/21/21 pairs (44/42/42 dims)
+ * at head_dim 128, base 10000. */
+typedef struct {
+    int grid_h, grid_w;
+    int pairs_t, pairs_h, pairs_w;
+    double base;
+} kvcr_rope;
+
+/* MoBA training sequence [C1..Cn | N1..Nn | B], each C/N chunk chunk_tokens long
+ * and B n_bidir_chunks * chunk_tokens long.  Mask: a query of C_i reads C_j for
+ * j <= i; a query of N_i reads C_j for j < i and N_i; a query of B reads B. */
+typedef struct {
+    int n_chunks;
+    int chunk_tokens;
+    int n_bidir_chunks;
+} kvcr_moba_layout;
+
+/* Tile classes returned by moba_classify_tiles. */
+enum { KVCR_TILE_EMPTY = 0, KVCR_TILE_PARTIAL = 1, KVCR_TILE_FULL = 2 };
+
+typedef struct kvcr_cache kvcr_cache;
+
+/* ---------------------------------------------------------------- cache --- */
+
+/* Bytes of device storage a cache needs: K and V of sinks+window frame slots,
+ * and, when with_rope != 0, scratch for the rotated queries and current-chunk
+ * keys of one chunk (chunk_frames frames) plus the (h, w) angle tables.
+ * Returns 0 for invalid sizes. */
+size_t kv_cache_storage_bytes(int sinks, int window, int tokens_per_frame, int heads,
+                              int head_dim, int chunk_frames, int with_rope,
+                              kvcr_dtype dtype);
+
+/* Create a cache.  sinks anchor slots + window recent slots; frames of
+ * tokens_per_frame tokens; heads x head_dim per token; chunk_frames = most
+ * frames in one current chunk.  rope = NULL disables rotary embedding (keys and
+ * queries are used as given, e.g. for text cross-attention).  device_storage /
+ * storage_bytes: a caller-owned device buffer (>= kv_cache_storage_bytes, 256-
+ * byte aligned) that must outlive the cache; the library writes the angle
+ * tables into it here (synchronously).  device_storage = NULL with
+ * storage_bytes = 0 creates a bookkeeping-only cache: the slot table works,
+ * kv_cache_append_rope() must then be given k = v = NULL and launches nothing,
+ * and attention calls return KVCR_ESTATE.  Supported: bf16 with head_dim 64 or
+ * 128 (tensor-core path), fp32 with head_dim 64 or 128 (fp32 CUDA-core path);
+ * sinks + window <= 32.  *out receives the handle. */
+int kv_cache_init(kvcr_cache **out, int sinks, int window, int tokens_per_frame, int heads,
+                  int head_dim, int chunk_frames, const kvcr_rope *rope, kvcr_dtype dtype,
+                  void *device_storage, size_t storage_bytes);
+
+/* Append finalized frames (the last denoising step's K and V).
+ * k, v: device [n_frames * tokens_per_frame][heads][head_dim].  frame_idx: host,
+ * n_frames strictly increasing absolute latent-frame indices, each larger than
+ * every frame appended before.  Frame by frame: an unfilled anchor slot is taken
+ * first; else, when the window holds `window` frames, the oldest non-anchor
+ * frame is evicted and its slot reused; else the lowest free window slot is
+ * taken.  K is written rotated (RoPE3D at its absolute (t, h, w)), V as is.
+ * A frame evicted by a later frame of the same call is not written.
+ * n_frames = 0 is a no-op. */
+int kv_cache_append_rope(kvcr_cache *c, const void *k, const void *v,
+                         const int32_t *frame_idx, int n_frames, void *stream);
+
+/* Dynamic window: evict the oldest non-anchor frames until at most keep_recent
+ * remain (0 <= keep_recent <= window).  Host only.  evicted_out (nullable) receives
+ * up to evicted_cap evicted frame indices, oldest first; *n_evicted (nullable)
+ * the number evicted. */
+int kv_cache_evict(kvcr_cache *c, int keep_recent, int32_t *evicted_out, int evicted_cap,
+                   int *n_evicted);
+
+/* Slot table: frame_of_slot[s] = frame cached in slot s or -1, s < sinks+window. */
+int kv_cache_slot_map(const kvcr_cache *c, int32_t *frame_of_slot, int cap);
+
+/* Result of the last append: slot of each appended frame (-1 = not retained)
+ * and the frames it evicted (oldest first). */
+int kv_cache_last_append(const kvcr_cache *c, int32_t *slots, int slots_cap,
+                         int32_t *evicted, int evicted_cap, int *n_evicted);
+
+/* Number of cached frames. */
+int kv_cache_num_cached(const kvcr_cache *c, int *n);
+
+/* Device addresses of slot `slot`'s K and V, each [tokens_per_frame][heads][head_dim]
+ * in the cache dtype (K stored rotated).  For reading back or saving a cache. */
+int kv_cache_slot_data(const kvcr_cache *c, int slot, const void **k, const void **v);
+
+void kv_cache_destroy(kvcr_cache *c);
+
+/* ------------------------------------------------------------ attention --- */
+
+/* Chunk attention: O = softmax(scale * Q K^T) V where the keys are every cached
+ * frame (anchors and window) followed by the current chunk's own n_cur_frames
+ * frames; full attention inside the chunk.
+ *   q:     device [n_q][heads][head_dim]; with RoPE, n_q must equal
+ *          n_cur_frames * tokens_per_frame (the chunk's tokens) and Q is rotated
+ *          at the chunk's positions; without RoPE n_q is free (cross-attention).
+ *   k_cur, v_cur: device [n_cur_frames * tokens_per_frame][heads][head_dim].
+ *   cur_frame_idx: host, strictly increasing, larger than every cached frame.
+ *   softmax_scale <= 0 means 1/sqrt(head_dim).
+ *   o:     device [n_q][heads][head_dim] in the cache dtype.
+ *   lse:   nullable device fp32 [heads][n_q], natural-log sum of exp of scores.
+ * The cache is read, not changed. */
+int chunk_attention_fwd(kvcr_cache *c, const void *q, int n_q, const void *k_cur,
+                        const void *v_cur, const int32_t *cur_frame_idx, int n_cur_frames,
+                        float softmax_scale, void *o, float *lse, void *stream);
+
+/* Attention under the MoBA mask over one sequence of L = layout tokens.
+ * q, k, v, o: device [L][heads][head_dim] bf16 (head_dim 128 or 64); lse nullable
+ * fp32 [heads][L].  128 x 128 tiles of the score matrix with no allowed entry
+ * are skipped, fully allowed tiles run unmasked, the rest are masked. */
+int moba_attention_fwd(const void *q, const void *k, const void *v,
+                       const kvcr_moba_layout *layout, int heads, int head_dim,
+                       kvcr_dtype dtype, float softmax_scale, void *o, float *lse,
+                       void *stream);
+
+/* Host classification of the tile x tile blocks of the MoBA score matrix into
+ * KVCR_TILE_EMPTY / PARTIAL / FULL (only in-range rows and columns count).
+ * cls: host [nt * nt] row-major, nt = ceil(L / tile); cap = its length. */
+int moba_classify_tiles(const kvcr_moba_layout *layout, int tile, uint8_t *cls, size_t cap);
+
+/* ------------------------------------------------------------- status ---- */
+
+/* Synchronise `stream` and return (then clear) the device-side status of the
+ * library's kernels on the current device: KVCR_OK or KVCR_ETIMEOUT when a
+ * kernel gave up on a bounded wait (its outputs are then invalid). */
+int kvcr_check_status(void *stream);
+
+const char *kvcr_last_error(void);
+
+/* -------------------------------------------------------------- trace ---- */
+
+/* Kernel ids for tracing. */
+enum {
+    KVCR_K_APPEND_ROPE = 0, /* cache write: RoPE3D(K) + copy V into slots */
+    KVCR_K_ROPE_STAGE = 1,  /* RoPE3D of the current chunk's Q and K into scratch */
+    KVCR_K_CHUNK_ATTN = 2,  /* tensor-core chunk attention (bf16) */
+    KVCR_K_MOBA_ATTN = 3,   /* tensor-core MoBA attention (bf16) */
+    KVCR_K_ATTN_F32 = 4,    /* fp32 CUDA-core attention */
+    KVCR_K_COUNT = 5
+};
+
+/* Count of every kernel the library launched in this process. */
+long long kvcr_launch_count(void);
+
+/* Tracing: when on, each launch is bracketed by two CUDA events recorded on
+ * its own stream.  kvcr_trace_reset() clears the records;
+ * kvcr_trace_read() waits for the recorded events and returns, for one kernel
+ * id, the number of traced launches and their summed device time in ms. */
+int kvcr_trace_enable(int on);
+int kvcr_trace_reset(void);
+int kvcr_trace_read(int kernel_id, long long *launches, double *total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVCR_H */

@@ -1,0 +1,823 @@
+// Host side of the C ABI declared in include/kvcr.h: argument validation, the
+// per-layer slot table (anchors + sliding window), device-storage layout,
+// rotary angle tables, TMA tensor-map encoding, kernel launches and tracing.
+//
+// Slot rules ("LingBot-World-Infinity: The Open-Source World Model That
+// Refuses to Forget", "The trick: treat video like a causal stream" and "How
+// the cache keeps the world alive"; "Westlake AGI Lab's 'World in World'
+// Steers Frozen Video Models", second paragraph):
+//   - the first `sinks` finalized frames are the anchors, slot i for the i-th;
+//     anchors are never evicted;
+//   - a later frame that finds `window` non-anchor frames cached evicts the
+//     oldest of them and takes its slot, else it takes the lowest free window
+//     slot;
+//   - kv_cache_evict(keep) drops the oldest non-anchor frames down to `keep`
+//     (the dynamic KV-cache scheduler of "Infinite Worlds with Versatile
+//     Interactions", deployment paragraph).
+// Bookkeeping never reads device memory, so every call stays asynchronous.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <deque>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "kvcr_internal.h"
+#include "moba_layout.h"
+
+using namespace kvcr;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const std::string& msg) {
+  g_err = msg;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(KVCR_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------ tensor maps --
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tiled map over a bf16 tensor [..][tokens][H][D] (innermost first: D, H,
+// tokens[, slots]); box = 64 x 1 x 128 (x 1), 128-byte swizzle, zero fill.
+int encode_bf16_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(KVCR_ECUDA, "cuTensorMapEncodeTiled not available from the driver");
+  cuuint64_t gdim[4];
+  cuuint64_t gstride[3];
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)kTile, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  uint64_t stride = 2;
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    if (i > 0) gstride[i - 1] = stride;
+    stride *= dims[i];
+  }
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KVCR_ECUDA, "cuTensorMapEncodeTiled failed (" +
+                                                     std::to_string((int)r) + ")");
+  return KVCR_OK;
+}
+
+// ----------------------------------------------------------------- tracing --
+std::atomic<long long> g_launches{0};
+std::mutex g_trace_mu;
+bool g_trace_on = false;
+struct TraceRec {
+  int kid;
+  cudaEvent_t a, b;
+};
+std::vector<TraceRec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t pool_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Brackets one launch with events on its stream when tracing is on.
+class LaunchScope {
+ public:
+  LaunchScope(int kid, cudaStream_t s) : kid_(kid), s_(s) {
+    g_launches.fetch_add(1);
+    std::lock_guard<std::mutex> g(g_trace_mu);
+    if (g_trace_on) {
+      a_ = pool_event();
+      b_ = pool_event();
+      if (a_ && b_) cudaEventRecord(a_, s_);
+    }
+  }
+  ~LaunchScope() {
+    if (!a_ || !b_) return;
+    cudaEventRecord(b_, s_);
+    std::lock_guard<std::mutex> g(g_trace_mu);
+    g_recs.push_back({kid_, a_, b_});
+  }
+
+ private:
+  int kid_;
+  cudaStream_t s_;
+  cudaEvent_t a_ = nullptr, b_ = nullptr;
+};
+
+// -------------------------------------------------------------- device info --
+int device_sm_count(int* n_sm, int* cc_major) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  e = cudaDeviceGetAttribute(n_sm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  e = cudaDeviceGetAttribute(cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  return KVCR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct StorageLayout {
+  size_t k_off, v_off, q_off, ks_off, h_off, w_off, total;
+};
+
+bool make_layout(int S, int W, int T, int H, int D, int F, bool rope, size_t esize,
+                 StorageLayout* L) {
+  if (S < 0 || W < 0 || S + W < 1 || S + W > kMaxSlots || T < 1 || H < 1 || D < 1 || F < 1 ||
+      F > kMaxFrames)
+    return false;
+  const size_t frame = (size_t)T * H * D * esize;
+  const size_t slots = (size_t)(S + W);
+  size_t off = 0;
+  L->k_off = off;
+  off = align_up(off + slots * frame, 256);
+  L->v_off = off;
+  off = align_up(off + slots * frame, 256);
+  L->q_off = L->ks_off = L->h_off = L->w_off = off;
+  if (rope) {
+    L->q_off = off;
+    off = align_up(off + (size_t)F * frame, 256);
+    L->ks_off = off;
+    off = align_up(off + (size_t)F * frame, 256);
+    // angle tables: at most T rows x D/2 pairs each for h and w
+    L->h_off = off;
+    off = align_up(off + (size_t)T * (D / 2) * sizeof(float2), 256);
+    L->w_off = off;
+    off = align_up(off + (size_t)T * (D / 2) * sizeof(float2), 256);
+  }
+  L->total = off;
+  return true;
+}
+
+}  // namespace
+
+// ====================================================================== cache
+struct kvcr_cache {
+  int S, W, T, H, D, F;
+  kvcr_dtype dtype;
+  size_t esize;
+  bool rope;
+  kvcr_rope rp;
+  bool has_storage;
+  uint8_t* storage;
+  StorageLayout lay;
+  int n_sm, cc_major;
+  CUtensorMap tm_kc, tm_vc;
+  // slot table
+  std::vector<int> slot_frame;
+  int n_sinks_filled;
+  std::deque<int> recent;  // non-anchor frames, oldest first
+  int last_frame;
+  std::vector<int> last_slots, last_evicted;
+};
+
+namespace {
+
+struct SlotState {
+  std::vector<int> slot_frame;
+  int n_sinks_filled;
+  std::deque<int> recent;
+  int last_frame;
+};
+
+SlotState snapshot(const kvcr_cache* c) {
+  return SlotState{c->slot_frame, c->n_sinks_filled, c->recent, c->last_frame};
+}
+
+void restore(kvcr_cache* c, const SlotState& s) {
+  c->slot_frame = s.slot_frame;
+  c->n_sinks_filled = s.n_sinks_filled;
+  c->recent = s.recent;
+  c->last_frame = s.last_frame;
+}
+
+// Apply the slot rules to one frame; returns its slot (-1 = not retained) and
+// appends evicted frames.
+int place_frame(kvcr_cache* c, int f, std::vector<int>& evicted) {
+  int s;
+  c->last_frame = f;
+  if (c->n_sinks_filled < c->S) {
+    s = c->n_sinks_filled++;
+  } else if (c->W == 0) {
+    evicted.push_back(f);
+    return -1;
+  } else if ((int)c->recent.size() == c->W) {
+    const int old = c->recent.front();
+    c->recent.pop_front();
+    s = -1;
+    for (int i = c->S; i < c->S + c->W; ++i)
+      if (c->slot_frame[i] == old) s = i;
+    c->slot_frame[s] = -1;
+    evicted.push_back(old);
+    c->recent.push_back(f);
+  } else {
+    s = -1;
+    for (int i = c->S; i < c->S + c->W && s < 0; ++i)
+      if (c->slot_frame[i] == -1) s = i;
+    c->recent.push_back(f);
+  }
+  c->slot_frame[s] = f;
+  return s;
+}
+
+void fill_ttab(const kvcr_cache* c, RopeCopyParams& p, const int32_t* frames, int n) {
+  for (int f = 0; f < n; ++f)
+    for (int j = 0; j < c->rp.pairs_t; ++j) {
+      const double ang =
+          (double)frames[f] * std::pow(c->rp.base, -(2.0 * j) / (2.0 * c->rp.pairs_t));
+      p.ttab[f][j] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
+}
+
+void fill_common(const kvcr_cache* c, RopeCopyParams& p) {
+  p.T = c->T;
+  p.H = c->H;
+  p.D = c->D;
+  p.grid_w = c->rope ? c->rp.grid_w : 1;
+  p.pairs_t = c->rope ? c->rp.pairs_t : 0;
+  p.pairs_h = c->rope ? c->rp.pairs_h : 0;
+  p.pairs_w = c->rope ? c->rp.pairs_w : 0;
+  p.htab = c->rope ? reinterpret_cast<const float2*>(c->storage + c->lay.h_off) : nullptr;
+  p.wtab = c->rope ? reinterpret_cast<const float2*>(c->storage + c->lay.w_off) : nullptr;
+}
+
+int check_frames(const kvcr_cache* c, const int32_t* frames, int n, const char* what) {
+  if (n > 0 && frames == nullptr) return fail(KVCR_EINVAL, std::string(what) + ": frame indices are NULL");
+  int prev = c->last_frame;
+  for (int i = 0; i < n; ++i) {
+    if (frames[i] < 0) return fail(KVCR_EINVAL, std::string(what) + ": negative frame index");
+    if (frames[i] <= prev)
+      return fail(KVCR_ESTATE, std::string(what) +
+                                   ": frame indices must increase and exceed every cached frame");
+    prev = frames[i];
+  }
+  return KVCR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvcr_last_error(void) { return g_err.c_str(); }
+
+size_t kv_cache_storage_bytes(int sinks, int window, int tokens_per_frame, int heads, int head_dim,
+                              int chunk_frames, int with_rope, kvcr_dtype dtype) {
+  if (dtype != KVCR_BF16 && dtype != KVCR_F32) return 0;
+  StorageLayout L;
+  if (!make_layout(sinks, window, tokens_per_frame, heads, head_dim, chunk_frames, with_rope != 0,
+                   dtype == KVCR_BF16 ? 2 : 4, &L))
+    return 0;
+  return L.total;
+}
+
+int kv_cache_init(kvcr_cache** out, int sinks, int window, int tokens_per_frame, int heads,
+                  int head_dim, int chunk_frames, const kvcr_rope* rope, kvcr_dtype dtype,
+                  void* device_storage, size_t storage_bytes) {
+  if (out == nullptr) return fail(KVCR_EINVAL, "kv_cache_init: out is NULL");
+  *out = nullptr;
+  if (dtype != KVCR_BF16 && dtype != KVCR_F32) return fail(KVCR_EINVAL, "kv_cache_init: bad dtype");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(KVCR_EUNSUPPORTED, "kv_cache_init: head_dim must be 64 or 128");
+  if (sinks < 0 || window < 0 || sinks + window < 1 || sinks + window > kMaxSlots)
+    return fail(KVCR_ESHAPE, "kv_cache_init: need 1 <= sinks + window <= 32");
+  if (tokens_per_frame < 1 || heads < 1 || chunk_frames < 1 || chunk_frames > kMaxFrames)
+    return fail(KVCR_ESHAPE, "kv_cache_init: bad tokens_per_frame / heads / chunk_frames (<= 16)");
+  if ((long long)chunk_frames * tokens_per_frame > (1LL << 30) ||
+      (long long)tokens_per_frame * heads * head_dim > (1LL << 31) / 4)
+    return fail(KVCR_ESHAPE, "kv_cache_init: frame too large");
+  if (rope) {
+    if ((long long)rope->grid_h * rope->grid_w != tokens_per_frame || rope->grid_h < 1 ||
+        rope->grid_w < 1)
+      return fail(KVCR_ESHAPE, "kv_cache_init: rope grid_h * grid_w != tokens_per_frame");
+    if (rope->pairs_t < 0 || rope->pairs_h < 0 || rope->pairs_w < 0 ||
+        rope->pairs_t + rope->pairs_h + rope->pairs_w != head_dim / 2 ||
+        rope->pairs_t > kMaxPairsT)
+      return fail(KVCR_ESHAPE, "kv_cache_init: rope pairs must sum to head_dim/2 (pairs_t <= 32)");
+    if (!(rope->base > 0.0)) return fail(KVCR_EINVAL, "kv_cache_init: rope base must be > 0");
+  }
+  const size_t esize = dtype == KVCR_BF16 ? 2 : 4;
+  StorageLayout L;
+  if (!make_layout(sinks, window, tokens_per_frame, heads, head_dim, chunk_frames, rope != nullptr,
+                   esize, &L))
+    return fail(KVCR_ESHAPE, "kv_cache_init: bad sizes");
+  const bool has_storage = device_storage != nullptr;
+  if (!has_storage && storage_bytes != 0)
+    return fail(KVCR_ESTORAGE, "kv_cache_init: storage is NULL but storage_bytes != 0");
+  int n_sm = 0, cc = 0;
+  if (has_storage) {
+    if (storage_bytes < L.total)
+      return fail(KVCR_ESTORAGE, "kv_cache_init: storage smaller than kv_cache_storage_bytes()");
+    if ((reinterpret_cast<uintptr_t>(device_storage) & 255u) != 0)
+      return fail(KVCR_ESTORAGE, "kv_cache_init: storage must be 256-byte aligned");
+    int rc = device_sm_count(&n_sm, &cc);
+    if (rc) return rc;
+    if (dtype == KVCR_BF16 && cc != 10)
+      return fail(KVCR_EUNSUPPORTED, "kv_cache_init: the bf16 path needs an sm_100 GPU");
+  }
+  kvcr_cache* c = new kvcr_cache();
+  c->S = sinks;
+  c->W = window;
+  c->T = tokens_per_frame;
+  c->H = heads;
+  c->D = head_dim;
+  c->F = chunk_frames;
+  c->dtype = dtype;
+  c->esize = esize;
+  c->rope = rope != nullptr;
+  if (rope) c->rp = *rope;
+  c->has_storage = has_storage;
+  c->storage = static_cast<uint8_t*>(device_storage);
+  c->lay = L;
+  c->n_sm = n_sm;
+  c->cc_major = cc;
+  c->slot_frame.assign(sinks + window, -1);
+  c->n_sinks_filled = 0;
+  c->last_frame = -1;
+  if (has_storage) {
+    if (c->rope) {
+      // (h, w) angle tables in double precision, stored as fp32 (cos, sin).
+      std::vector<float2> ht((size_t)rope->grid_h * std::max(rope->pairs_h, 1));
+      std::vector<float2> wt((size_t)rope->grid_w * std::max(rope->pairs_w, 1));
+      for (int y = 0; y < rope->grid_h; ++y)
+        for (int j = 0; j < rope->pairs_h; ++j) {
+          const double a = (double)y * std::pow(rope->base, -(2.0 * j) / (2.0 * rope->pairs_h));
+          ht[(size_t)y * rope->pairs_h + j] = make_float2((float)std::cos(a), (float)std::sin(a));
+        }
+      for (int x = 0; x < rope->grid_w; ++x)
+        for (int j = 0; j < rope->pairs_w; ++j) {
+          const double a = (double)x * std::pow(rope->base, -(2.0 * j) / (2.0 * rope->pairs_w));
+          wt[(size_t)x * rope->pairs_w + j] = make_float2((float)std::cos(a), (float)std::sin(a));
+        }
+      cudaError_t e = cudaMemcpy(c->storage + L.h_off, ht.data(), ht.size() * sizeof(float2),
+                                 cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(c->storage + L.w_off, wt.data(), wt.size() * sizeof(float2),
+                       cudaMemcpyHostToDevice);
+      if (e != cudaSuccess) {
+        delete c;
+        return cuda_fail(e, "kv_cache_init: writing angle tables");
+      }
+    }
+    if (dtype == KVCR_BF16) {
+      const uint64_t dims[4] = {(uint64_t)head_dim, (uint64_t)heads, (uint64_t)tokens_per_frame,
+                                (uint64_t)(sinks + window)};
+      int rc = encode_bf16_map(&c->tm_kc, c->storage + L.k_off, 4, dims);
+      if (!rc) rc = encode_bf16_map(&c->tm_vc, c->storage + L.v_off, 4, dims);
+      if (rc) {
+        delete c;
+        return rc;
+      }
+    }
+  }
+  *out = c;
+  return KVCR_OK;
+}
+
+void kv_cache_destroy(kvcr_cache* c) { delete c; }
+
+int kv_cache_append_rope(kvcr_cache* c, const void* k, const void* v, const int32_t* frame_idx,
+                         int n_frames, void* stream) {
+  if (c == nullptr) return fail(KVCR_EINVAL, "kv_cache_append_rope: cache is NULL");
+  if (n_frames < 0 || n_frames > kMaxFrames)
+    return fail(KVCR_ESHAPE, "kv_cache_append_rope: n_frames must be in [0, 16]");
+  if (n_frames == 0) {
+    c->last_slots.clear();
+    c->last_evicted.clear();
+    return KVCR_OK;
+  }
+  int rc = check_frames(c, frame_idx, n_frames, "kv_cache_append_rope");
+  if (rc) return rc;
+  if (c->has_storage) {
+    if (k == nullptr || v == nullptr) return fail(KVCR_EINVAL, "kv_cache_append_rope: k/v NULL");
+    if (!aligned16(k) || !aligned16(v))
+      return fail(KVCR_EINVAL, "kv_cache_append_rope: k/v must be 16-byte aligned");
+  } else if (k != nullptr || v != nullptr) {
+    return fail(KVCR_ESTATE, "kv_cache_append_rope: bookkeeping-only cache takes k = v = NULL");
+  }
+  const SlotState before = snapshot(c);
+  std::vector<int> slots(n_frames), evicted;
+  for (int i = 0; i < n_frames; ++i) slots[i] = place_frame(c, frame_idx[i], evicted);
+  if (c->has_storage) {
+    RopeCopyParams p;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(c, p);
+    p.src_a = k;
+    p.src_b = v;
+    p.dst_a = c->storage + c->lay.k_off;
+    p.dst_b = c->storage + c->lay.v_off;
+    p.rotate_a = c->rope ? 1 : 0;
+    p.rotate_b = 0;
+    const long long frame_elems = (long long)c->T * c->H * c->D;
+    int n = 0;
+    std::vector<int32_t> written;
+    for (int i = 0; i < n_frames; ++i) {
+      // skip frames not retained, or evicted again by a later frame of this call
+      if (slots[i] < 0 || c->slot_frame[slots[i]] != frame_idx[i]) continue;
+      p.dst_frame_off[n] = (long long)slots[i] * frame_elems;
+      p.src_frame[n] = i;
+      written.push_back(frame_idx[i]);
+      ++n;
+    }
+    p.n_frames = n;
+    if (c->rope) fill_ttab(c, p, written.data(), n);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    {
+      LaunchScope scope(KVCR_K_APPEND_ROPE, s);
+      e = launch_rope_copy(p, c->dtype, s, c->n_sm);
+    }
+    if (e != cudaSuccess) {
+      restore(c, before);
+      return cuda_fail(e, "kv_cache_append_rope: launch");
+    }
+  }
+  c->last_slots = slots;
+  c->last_evicted = evicted;
+  return KVCR_OK;
+}
+
+int kv_cache_evict(kvcr_cache* c, int keep_recent, int32_t* evicted_out, int evicted_cap,
+                   int* n_evicted) {
+  if (c == nullptr) return fail(KVCR_EINVAL, "kv_cache_evict: cache is NULL");
+  if (keep_recent < 0 || keep_recent > c->W)
+    return fail(KVCR_EINVAL, "kv_cache_evict: keep_recent must be in [0, window]");
+  int n = 0;
+  while ((int)c->recent.size() > keep_recent) {
+    const int old = c->recent.front();
+    c->recent.pop_front();
+    for (int i = c->S; i < c->S + c->W; ++i)
+      if (c->slot_frame[i] == old) c->slot_frame[i] = -1;
+    if (evicted_out && n < evicted_cap) evicted_out[n] = old;
+    ++n;
+  }
+  if (n_evicted) *n_evicted = n;
+  return KVCR_OK;
+}
+
+int kv_cache_slot_map(const kvcr_cache* c, int32_t* frame_of_slot, int cap) {
+  if (c == nullptr || frame_of_slot == nullptr) return fail(KVCR_EINVAL, "kv_cache_slot_map: NULL");
+  if (cap < c->S + c->W) return fail(KVCR_ESHAPE, "kv_cache_slot_map: cap < sinks + window");
+  for (int i = 0; i < c->S + c->W; ++i) frame_of_slot[i] = c->slot_frame[i];
+  return KVCR_OK;
+}
+
+int kv_cache_last_append(const kvcr_cache* c, int32_t* slots, int slots_cap, int32_t* evicted,
+                         int evicted_cap, int* n_evicted) {
+  if (c == nullptr) return fail(KVCR_EINVAL, "kv_cache_last_append: NULL");
+  if (slots)
+    for (int i = 0; i < (int)c->last_slots.size() && i < slots_cap; ++i) slots[i] = c->last_slots[i];
+  if (evicted)
+    for (int i = 0; i < (int)c->last_evicted.size() && i < evicted_cap; ++i)
+      evicted[i] = c->last_evicted[i];
+  if (n_evicted) *n_evicted = (int)c->last_evicted.size();
+  return KVCR_OK;
+}
+
+int kv_cache_num_cached(const kvcr_cache* c, int* n) {
+  if (c == nullptr || n == nullptr) return fail(KVCR_EINVAL, "kv_cache_num_cached: NULL");
+  int k = 0;
+  for (int f : c->slot_frame) k += f >= 0;
+  *n = k;
+  return KVCR_OK;
+}
+
+int kv_cache_slot_data(const kvcr_cache* c, int slot, const void** k, const void** v) {
+  if (c == nullptr || k == nullptr || v == nullptr)
+    return fail(KVCR_EINVAL, "kv_cache_slot_data: NULL");
+  if (!c->has_storage) return fail(KVCR_ESTATE, "kv_cache_slot_data: bookkeeping-only cache");
+  if (slot < 0 || slot >= c->S + c->W) return fail(KVCR_EINVAL, "kv_cache_slot_data: bad slot");
+  const size_t frame = (size_t)c->T * c->H * c->D * c->esize;
+  *k = c->storage + c->lay.k_off + (size_t)slot * frame;
+  *v = c->storage + c->lay.v_off + (size_t)slot * frame;
+  return KVCR_OK;
+}
+
+int chunk_attention_fwd(kvcr_cache* c, const void* q, int n_q, const void* k_cur,
+                        const void* v_cur, const int32_t* cur_frame_idx, int n_cur_frames,
+                        float softmax_scale, void* o, float* lse, void* stream) {
+  if (c == nullptr) return fail(KVCR_EINVAL, "chunk_attention_fwd: cache is NULL");
+  if (!c->has_storage) return fail(KVCR_ESTATE, "chunk_attention_fwd: bookkeeping-only cache");
+  if (n_cur_frames < 1 || n_cur_frames > c->F)
+    return fail(KVCR_ESHAPE, "chunk_attention_fwd: n_cur_frames must be in [1, chunk_frames]");
+  if (n_q < 0) return fail(KVCR_ESHAPE, "chunk_attention_fwd: n_q < 0");
+  const int n_cur = n_cur_frames * c->T;
+  if (c->rope && n_q != n_cur)
+    return fail(KVCR_ESHAPE, "chunk_attention_fwd: with RoPE n_q must be n_cur_frames * T");
+  int rc = check_frames(c, cur_frame_idx, n_cur_frames, "chunk_attention_fwd");
+  if (rc) return rc;
+  if (n_q == 0) return KVCR_OK;
+  if (!q || !k_cur || !v_cur || !o) return fail(KVCR_EINVAL, "chunk_attention_fwd: NULL tensor");
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(o))
+    return fail(KVCR_EINVAL, "chunk_attention_fwd: tensors must be 16-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(KVCR_EINVAL, "chunk_attention_fwd: lse must be 4-byte aligned");
+  if ((long long)n_q * c->H * c->D > (1LL << 31) - 1)
+    return fail(KVCR_ESHAPE, "chunk_attention_fwd: n_q too large");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)c->D);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // visible cached frames, in slot order
+  int slots[kMaxSlots];
+  int n_vis = 0;
+  for (int i = 0; i < c->S + c->W; ++i)
+    if (c->slot_frame[i] >= 0) slots[n_vis++] = i;
+
+  const void* q_src = q;
+  const void* k_src = k_cur;
+  if (c->rope) {
+    RopeCopyParams p;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(c, p);
+    p.src_a = q;
+    p.src_b = k_cur;
+    p.dst_a = c->storage + c->lay.q_off;
+    p.dst_b = c->storage + c->lay.ks_off;
+    p.rotate_a = 1;
+    p.rotate_b = 1;
+    p.n_frames = n_cur_frames;
+    const long long frame_elems = (long long)c->T * c->H * c->D;
+    for (int f = 0; f < n_cur_frames; ++f) {
+      p.dst_frame_off[f] = f * frame_elems;
+      p.src_frame[f] = f;
+    }
+    fill_ttab(c, p, cur_frame_idx, n_cur_frames);
+    cudaError_t e;
+    {
+      LaunchScope scope(KVCR_K_ROPE_STAGE, s);
+      e = launch_rope_copy(p, c->dtype, s, c->n_sm);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd: rope stage launch");
+    q_src = c->storage + c->lay.q_off;
+    k_src = c->storage + c->lay.ks_off;
+  }
+
+  if (c->dtype == KVCR_BF16) {
+    ChunkAttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t dq[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_q};
+    const uint64_t dn[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_cur};
+    rc = encode_bf16_map(&p.tm_q, q_src, 3, dq);
+    if (!rc) rc = encode_bf16_map(&p.tm_kn, k_src, 3, dn);
+    if (!rc) rc = encode_bf16_map(&p.tm_vn, v_cur, 3, dn);
+    if (rc) return rc;
+    p.tm_kc = c->tm_kc;
+    p.tm_vc = c->tm_vc;
+    p.c.o = o;
+    p.c.lse = lse;
+    p.c.n_q = n_q;
+    p.c.H = c->H;
+    p.c.scale_log2 = (float)(scale * 1.4426950408889634);
+    p.s.T = c->T;
+    p.s.n_vis = n_vis;
+    p.s.tiles_per_slot = (c->T + kTile - 1) / kTile;
+    p.s.n_cur = n_cur;
+    p.s.cur_tiles = (n_cur + kTile - 1) / kTile;
+    for (int i = 0; i < n_vis; ++i) p.s.slots[i] = slots[i];
+    cudaError_t e;
+    {
+      LaunchScope scope(KVCR_K_CHUNK_ATTN, s);
+      e = launch_chunk_attn_sm100(p, c->D, (n_q + kTile - 1) / kTile, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd: attention launch");
+  } else {
+    F32AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = static_cast<const float*>(q_src);
+    p.kc = reinterpret_cast<const float*>(c->storage + c->lay.k_off);
+    p.vc = reinterpret_cast<const float*>(c->storage + c->lay.v_off);
+    p.kn = static_cast<const float*>(k_src);
+    p.vn = static_cast<const float*>(v_cur);
+    p.o = static_cast<float*>(o);
+    p.lse = lse;
+    p.n_q = n_q;
+    p.H = c->H;
+    p.D = c->D;
+    p.T = c->T;
+    p.n_vis = n_vis;
+    p.n_cur = n_cur;
+    p.scale = scale;
+    for (int i = 0; i < n_vis; ++i) p.slots[i] = slots[i];
+    cudaError_t e;
+    {
+      LaunchScope scope(KVCR_K_ATTN_F32, s);
+      e = launch_attn_f32(p, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd: fp32 attention launch");
+  }
+  return KVCR_OK;
+}
+
+// ======================================================================= MoBA
+static int moba_check_layout(const kvcr_moba_layout* layout, MobaLay* out) {
+  if (layout == nullptr) return fail(KVCR_EINVAL, "moba: layout is NULL");
+  if (layout->n_chunks < 1 || layout->chunk_tokens < 1 || layout->n_bidir_chunks < 0)
+    return fail(KVCR_ESHAPE, "moba: need n_chunks >= 1, chunk_tokens >= 1, n_bidir_chunks >= 0");
+  const long long L =
+      (2LL * layout->n_chunks + layout->n_bidir_chunks) * (long long)layout->chunk_tokens;
+  if (L > (long long)kMobaMaxTiles * kTile)
+    return fail(KVCR_ESHAPE, "moba: sequence longer than 4096 * 128 tokens");
+  *out = MobaLay{layout->n_chunks, layout->chunk_tokens, layout->n_bidir_chunks, (int)L};
+  return KVCR_OK;
+}
+
+int moba_classify_tiles(const kvcr_moba_layout* layout, int tile, uint8_t* cls, size_t cap) {
+  MobaLay l;
+  int rc = moba_check_layout(layout, &l);
+  if (rc) return rc;
+  if (tile < 1) return fail(KVCR_EINVAL, "moba_classify_tiles: tile < 1");
+  const long long nt = ((long long)l.L + tile - 1) / tile;
+  if (cls == nullptr || (long long)cap < nt * nt)
+    return fail(KVCR_ESHAPE, "moba_classify_tiles: output smaller than nt * nt");
+  for (long long i = 0; i < nt; ++i)
+    for (long long j = 0; j < nt; ++j)
+      cls[i * nt + j] = (uint8_t)moba_classify(l, (int)i, (int)j, tile);
+  return KVCR_OK;
+}
+
+namespace {
+// Non-empty key tiles of each 128-row tile (tiles hit by the union of the
+// rows' allowed key intervals), and the row tiles ordered heaviest first.
+void moba_order(const MobaLay& l, std::vector<uint16_t>& order) {
+  const int nt = (l.L + kTile - 1) / kTile;
+  std::vector<int> work(nt);
+  std::vector<std::pair<int, int>> iv;
+  int lo[2 * kTile + 8], hi[2 * kTile + 8];
+  for (int i = 0; i < nt; ++i) {
+    const int r0 = i * kTile, r1 = std::min(r0 + kTile, l.L);
+    const int n = moba_row_intervals(l, r0, r1, lo, hi, 2 * kTile + 8);
+    iv.clear();
+    for (int k = 0; k < n; ++k)
+      if (hi[k] > lo[k]) iv.push_back({lo[k] / kTile, (hi[k] - 1) / kTile});
+    std::sort(iv.begin(), iv.end());
+    int count = 0, cur_lo = -1, cur_hi = -2;
+    for (auto& t : iv) {
+      if (t.first > cur_hi) {
+        if (cur_hi >= cur_lo && cur_lo >= 0) count += cur_hi - cur_lo + 1;
+        cur_lo = t.first;
+        cur_hi = t.second;
+      } else {
+        cur_hi = std::max(cur_hi, t.second);
+      }
+    }
+    if (cur_lo >= 0) count += cur_hi - cur_lo + 1;
+    work[i] = count;
+  }
+  order.resize(nt);
+  for (int i = 0; i < nt; ++i) order[i] = (uint16_t)i;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](uint16_t a, uint16_t b) { return work[a] > work[b]; });
+}
+}  // namespace
+
+int moba_attention_fwd(const void* q, const void* k, const void* v,
+                       const kvcr_moba_layout* layout, int heads, int head_dim, kvcr_dtype dtype,
+                       float softmax_scale, void* o, float* lse, void* stream) {
+  MobaLay l;
+  int rc = moba_check_layout(layout, &l);
+  if (rc) return rc;
+  if (dtype != KVCR_BF16) return fail(KVCR_EUNSUPPORTED, "moba_attention_fwd: bf16 only");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(KVCR_EUNSUPPORTED, "moba_attention_fwd: head_dim must be 64 or 128");
+  if (heads < 1) return fail(KVCR_ESHAPE, "moba_attention_fwd: heads < 1");
+  if ((long long)l.L * heads * head_dim > (1LL << 31) - 1)
+    return fail(KVCR_ESHAPE, "moba_attention_fwd: tensor too large");
+  if (!q || !k || !v || !o) return fail(KVCR_EINVAL, "moba_attention_fwd: NULL tensor");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(KVCR_EINVAL, "moba_attention_fwd: tensors must be 16-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(KVCR_EINVAL, "moba_attention_fwd: lse must be 4-byte aligned");
+  int n_sm = 0, cc = 0;
+  rc = device_sm_count(&n_sm, &cc);
+  if (rc) return rc;
+  if (cc != 10) return fail(KVCR_EUNSUPPORTED, "moba_attention_fwd: needs an sm_100 GPU");
+
+  static std::mutex mu;
+  static MobaLay last{0, 0, 0, 0};
+  static std::vector<uint16_t> last_order;
+  MobaAttnParams* p = new MobaAttnParams();
+  std::memset(p, 0, sizeof(*p));
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (!(last.n == l.n && last.c == l.c && last.m == l.m)) {
+      moba_order(l, last_order);
+      last = l;
+    }
+    for (size_t i = 0; i < last_order.size(); ++i) p->s.order[i] = last_order[i];
+  }
+  const uint64_t d3[3] = {(uint64_t)head_dim, (uint64_t)heads, (uint64_t)l.L};
+  rc = encode_bf16_map(&p->tm_q, q, 3, d3);
+  if (!rc) rc = encode_bf16_map(&p->tm_k, k, 3, d3);
+  if (!rc) rc = encode_bf16_map(&p->tm_v, v, 3, d3);
+  if (rc) {
+    delete p;
+    return rc;
+  }
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)head_dim);
+  p->c.o = o;
+  p->c.lse = lse;
+  p->c.n_q = l.L;
+  p->c.H = heads;
+  p->c.scale_log2 = (float)(scale * 1.4426950408889634);
+  p->s.n_chunks = l.n;
+  p->s.chunk_tokens = l.c;
+  p->s.n_bidir = l.m;
+  p->s.L = l.L;
+  p->s.n_row_tiles = (l.L + kTile - 1) / kTile;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  {
+    LaunchScope scope(KVCR_K_MOBA_ATTN, s);
+    e = launch_moba_attn_sm100(*p, head_dim, s);
+  }
+  delete p;
+  if (e != cudaSuccess) return cuda_fail(e, "moba_attention_fwd: launch");
+  return KVCR_OK;
+}
+
+// ===================================================================== status
+int kvcr_check_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int a = 0, b = 0;
+  cudaError_t e = read_and_clear_status_attn(&a, s);
+  if (e == cudaSuccess) e = read_and_clear_status_f32(&b, s);
+  if (e != cudaSuccess) return cuda_fail(e, "kvcr_check_status");
+  if (a != 0 || b != 0) return fail(KVCR_ETIMEOUT, "a kernel gave up on a bounded wait");
+  return KVCR_OK;
+}
+
+long long kvcr_launch_count(void) { return g_launches.load(); }
+
+int kvcr_trace_enable(int on) {
+  std::lock_guard<std::mutex> g(g_trace_mu);
+  g_trace_on = on != 0;
+  return KVCR_OK;
+}
+
+int kvcr_trace_reset(void) {
+  std::lock_guard<std::mutex> g(g_trace_mu);
+  for (auto& r : g_recs) {
+    cudaEventSynchronize(r.b);
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_recs.clear();
+  return KVCR_OK;
+}
+
+int kvcr_trace_read(int kernel_id, long long* launches, double* total_ms) {
+  if (kernel_id < 0 || kernel_id >= KVCR_K_COUNT) return fail(KVCR_EINVAL, "kvcr_trace_read: id");
+  std::lock_guard<std::mutex> g(g_trace_mu);
+  long long n = 0;
+  double ms = 0.0;
+  for (auto& r : g_recs) {
+    if (r.kid != kernel_id) continue;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "kvcr_trace_read");
+    float t = 0.f;
+    e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "kvcr_trace_read");
+    ms += t;
+    ++n;
+  }
+  if (launches) *launches = n;
+  if (total_ms) *total_ms = ms;
+  return KVCR_OK;
+}
+
+}  // extern "C"

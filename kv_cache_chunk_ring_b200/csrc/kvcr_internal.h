@@ -1,0 +1,108 @@
+// Internal declarations shared by the host library and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kvcr.h"
+
+namespace kvcr {
+
+// ----------------------------------------------------------------- limits --
+constexpr int kMaxSlots = 32;        // sinks + window
+constexpr int kMaxFrames = 16;       // frames of one append / one current chunk
+constexpr int kMaxPairsT = 32;       // rotary pairs on the t axis
+constexpr int kTile = 128;           // rows / keys per attention tile
+constexpr int kMobaMaxTiles = 4096;  // MoBA sequence length <= 4096 * 128 tokens
+constexpr long long kWaitTimeoutNs = 2000000000LL;  // bounded device waits: 2 s
+
+// ------------------------------------------------------- rope / copy pass --
+// One launch moves n_frames frames of two tensors (a and b) of shape
+// [T][H][D] each from contiguous sources to per-frame destinations, rotating
+// a (and b when rotate_b) with the 3D rotary embedding.
+struct RopeCopyParams {
+  const void* src_a;
+  const void* src_b;
+  void* dst_a;
+  void* dst_b;
+  long long dst_frame_off[kMaxFrames];  // element offset of frame f's destination
+  int src_frame[kMaxFrames];            // which source frame feeds destination f
+  int n_frames, T, H, D, grid_w;
+  int rotate_a, rotate_b;
+  int pairs_t, pairs_h, pairs_w;
+  const float2* htab;                   // [grid_h][pairs_h] (cos, sin)
+  const float2* wtab;                   // [grid_w][pairs_w] (cos, sin)
+  float2 ttab[kMaxFrames][kMaxPairsT];  // per destination frame, t-axis (cos, sin)
+};
+
+cudaError_t launch_rope_copy(const RopeCopyParams& p, kvcr_dtype dtype, cudaStream_t s,
+                             int n_sm);
+
+// ------------------------------------------------------------- attention --
+struct ChunkSched {
+  int T;             // tokens per cached frame
+  int n_vis;         // cached frames read, in slot order
+  int tiles_per_slot;
+  int n_cur;         // current-chunk keys
+  int cur_tiles;
+  int slots[kMaxSlots];
+};
+
+struct MobaSched {
+  int n_chunks, chunk_tokens, n_bidir;
+  int L;
+  int n_row_tiles;
+  uint16_t order[kMobaMaxTiles];  // row tiles, heaviest first
+};
+
+struct AttnCommon {
+  void* o;
+  float* lse;
+  int n_q;
+  int H;
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+struct ChunkAttnParams {
+  CUtensorMap tm_q;   // 3D (D, H, n_q)
+  CUtensorMap tm_kc;  // 4D (D, H, T, slots) cached K
+  CUtensorMap tm_vc;  // 4D cached V
+  CUtensorMap tm_kn;  // 3D (D, H, n_cur) current K
+  CUtensorMap tm_vn;  // 3D current V
+  AttnCommon c;
+  ChunkSched s;
+};
+
+struct MobaAttnParams {
+  CUtensorMap tm_q;   // 3D (D, H, L)
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  AttnCommon c;
+  MobaSched s;
+};
+
+cudaError_t launch_chunk_attn_sm100(const ChunkAttnParams& p, int head_dim, int n_q_tiles,
+                                    cudaStream_t s);
+cudaError_t launch_moba_attn_sm100(const MobaAttnParams& p, int head_dim, cudaStream_t s);
+
+// fp32 CUDA-core attention over the same key sequence (cached slots + current)
+struct F32AttnParams {
+  const float* q;       // [n_q][H][D]
+  const float* kc;      // cache K area [slots][T][H][D]
+  const float* vc;
+  const float* kn;      // current K [n_cur][H][D]
+  const float* vn;
+  float* o;
+  float* lse;
+  int n_q, H, D, T, n_vis, n_cur;
+  float scale;
+  int slots[kMaxSlots];
+};
+cudaError_t launch_attn_f32(const F32AttnParams& p, cudaStream_t s);
+
+// device status words (one per kernel translation unit)
+cudaError_t read_and_clear_status_attn(int* st, cudaStream_t s);
+cudaError_t read_and_clear_status_f32(int* st, cudaStream_t s);
+
+}  // namespace kvcr

@@ -1,0 +1,321 @@
+"""Python binding of the C ABI in ``include/kvcr.h`` (ctypes, marshalling only).
+
+Every function here has the name of the C entry point it calls and only turns
+Python / torch arguments into pointers and sizes; all work runs in the
+library's CUDA kernels.  The library is the in-tree ``libkvcr.so`` built by
+``kv_cache_chunk_ring_b200.build``; importing a function that needs it raises
+when it is missing (there is no fallback).  torch is used for device memory
+and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import List, Optional, Sequence, Tuple
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkvcr.so")
+
+KVCR_OK, KVCR_EINVAL, KVCR_ESHAPE, KVCR_ESTATE = 0, -1, -2, -3
+KVCR_ECUDA, KVCR_ETIMEOUT, KVCR_ESTORAGE, KVCR_EUNSUPPORTED = -4, -5, -6, -7
+KVCR_BF16, KVCR_F32 = 0, 1
+KVCR_TILE_EMPTY, KVCR_TILE_PARTIAL, KVCR_TILE_FULL = 0, 1, 2
+(KVCR_K_APPEND_ROPE, KVCR_K_ROPE_STAGE, KVCR_K_CHUNK_ATTN, KVCR_K_MOBA_ATTN,
+ KVCR_K_ATTN_F32) = range(5)
+KERNEL_NAMES = {KVCR_K_APPEND_ROPE: "append_rope", KVCR_K_ROPE_STAGE: "rope_stage",
+                KVCR_K_CHUNK_ATTN: "chunk_attn", KVCR_K_MOBA_ATTN: "moba_attn",
+                KVCR_K_ATTN_F32: "attn_f32"}
+
+# every symbol include/kvcr.h declares
+EXPORTS = [
+    "kv_cache_storage_bytes", "kv_cache_init", "kv_cache_append_rope", "kv_cache_evict",
+    "kv_cache_slot_map", "kv_cache_last_append", "kv_cache_num_cached", "kv_cache_slot_data",
+    "kv_cache_destroy",
+    "chunk_attention_fwd", "moba_attention_fwd", "moba_classify_tiles", "kvcr_check_status",
+    "kvcr_last_error", "kvcr_launch_count", "kvcr_trace_enable", "kvcr_trace_reset",
+    "kvcr_trace_read",
+]
+
+
+class KvcrError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"kvcr status {code}: {msg}")
+        self.code = code
+
+
+class kvcr_rope(ctypes.Structure):
+    _fields_ = [("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int), ("pairs_t", ctypes.c_int),
+                ("pairs_h", ctypes.c_int), ("pairs_w", ctypes.c_int), ("base", ctypes.c_double)]
+
+
+class kvcr_moba_layout(ctypes.Structure):
+    _fields_ = [("n_chunks", ctypes.c_int), ("chunk_tokens", ctypes.c_int),
+                ("n_bidir_chunks", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libkvcr.so``; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m kv_cache_chunk_ring_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    c_int, c_p, c_sz, c_f = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    sig = {
+        "kv_cache_storage_bytes": (c_sz, [c_int] * 7 + [c_int]),
+        "kv_cache_init": (c_int, [ctypes.POINTER(c_p), c_int, c_int, c_int, c_int, c_int, c_int,
+                                  ctypes.POINTER(kvcr_rope), c_int, c_p, c_sz]),
+        "kv_cache_append_rope": (c_int, [c_p, c_p, c_p, i32p, c_int, c_p]),
+        "kv_cache_evict": (c_int, [c_p, c_int, i32p, c_int, ctypes.POINTER(c_int)]),
+        "kv_cache_slot_map": (c_int, [c_p, i32p, c_int]),
+        "kv_cache_last_append": (c_int, [c_p, i32p, c_int, i32p, c_int, ctypes.POINTER(c_int)]),
+        "kv_cache_num_cached": (c_int, [c_p, ctypes.POINTER(c_int)]),
+        "kv_cache_slot_data": (c_int, [c_p, c_int, ctypes.POINTER(c_p), ctypes.POINTER(c_p)]),
+        "kv_cache_destroy": (None, [c_p]),
+        "chunk_attention_fwd": (c_int, [c_p, c_p, c_int, c_p, c_p, i32p, c_int, c_f, c_p, c_p,
+                                        c_p]),
+        "moba_attention_fwd": (c_int, [c_p, c_p, c_p, ctypes.POINTER(kvcr_moba_layout), c_int,
+                                       c_int, c_int, c_f, c_p, c_p, c_p]),
+        "moba_classify_tiles": (c_int, [ctypes.POINTER(kvcr_moba_layout), c_int, c_p, c_sz]),
+        "kvcr_check_status": (c_int, [c_p]),
+        "kvcr_last_error": (ctypes.c_char_p, []),
+        "kvcr_launch_count": (ctypes.c_longlong, []),
+        "kvcr_trace_enable": (c_int, [c_int]),
+        "kvcr_trace_reset": (c_int, []),
+        "kvcr_trace_read": (c_int, [c_int, ctypes.POINTER(ctypes.c_longlong),
+                                    ctypes.POINTER(ctypes.c_double)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(rc: int) -> None:
+    if rc != KVCR_OK:
+        raise KvcrError(rc, lib().kvcr_last_error().decode())
+
+
+def _i32(seq: Sequence[int]):
+    arr = (ctypes.c_int32 * max(1, len(seq)))(*[int(x) for x in seq])
+    return arr
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _dtype_code(dtype) -> int:
+    import torch
+    if dtype in (torch.bfloat16, "bf16", KVCR_BF16):
+        return KVCR_BF16
+    if dtype in (torch.float32, "f32", KVCR_F32):
+        return KVCR_F32
+    raise ValueError(f"unsupported dtype {dtype}")
+
+
+# ---------------------------------------------------------------- C names ---
+
+def kv_cache_storage_bytes(sinks, window, tokens_per_frame, heads, head_dim, chunk_frames,
+                           with_rope, dtype) -> int:
+    return int(lib().kv_cache_storage_bytes(sinks, window, tokens_per_frame, heads, head_dim,
+                                            chunk_frames, int(bool(with_rope)),
+                                            _dtype_code(dtype)))
+
+
+def kv_cache_init(sinks, window, tokens_per_frame, heads, head_dim, chunk_frames, rope, dtype,
+                  storage) -> ctypes.c_void_p:
+    """Create a cache over ``storage`` (a CUDA tensor, or None for bookkeeping only)."""
+    h = ctypes.c_void_p()
+    rp = None
+    if rope is not None:
+        rp = ctypes.byref(kvcr_rope(rope.grid_h, rope.grid_w, rope.pairs_t, rope.pairs_h,
+                                    rope.pairs_w, float(rope.base)))
+    ptr = None if storage is None else storage.data_ptr()
+    nbytes = 0 if storage is None else storage.numel() * storage.element_size()
+    _check(lib().kv_cache_init(ctypes.byref(h), sinks, window, tokens_per_frame, heads, head_dim,
+                               chunk_frames, rp, _dtype_code(dtype), ptr, nbytes))
+    return h
+
+
+def kv_cache_append_rope(handle, k, v, frame_idx: Sequence[int], stream=None) -> None:
+    n = len(frame_idx)
+    s = None if (k is None and v is None) else _stream(stream)
+    _check(lib().kv_cache_append_rope(handle, _ptr(k), _ptr(v), _i32(frame_idx), n, s))
+
+
+def kv_cache_evict(handle, keep_recent: int) -> List[int]:
+    buf = (ctypes.c_int32 * 64)()
+    n = ctypes.c_int()
+    _check(lib().kv_cache_evict(handle, keep_recent, buf, 64, ctypes.byref(n)))
+    return [int(buf[i]) for i in range(min(n.value, 64))]
+
+
+def kv_cache_slot_map(handle, n_slots: int) -> List[int]:
+    buf = (ctypes.c_int32 * n_slots)()
+    _check(lib().kv_cache_slot_map(handle, buf, n_slots))
+    return [int(x) for x in buf]
+
+
+def kv_cache_last_append(handle, n_frames: int) -> Tuple[List[int], List[int]]:
+    sl = (ctypes.c_int32 * max(1, n_frames))()
+    ev = (ctypes.c_int32 * 64)()
+    n = ctypes.c_int()
+    _check(lib().kv_cache_last_append(handle, sl, n_frames, ev, 64, ctypes.byref(n)))
+    return [int(sl[i]) for i in range(n_frames)], [int(ev[i]) for i in range(min(n.value, 64))]
+
+
+def kv_cache_num_cached(handle) -> int:
+    n = ctypes.c_int()
+    _check(lib().kv_cache_num_cached(handle, ctypes.byref(n)))
+    return n.value
+
+
+def kv_cache_slot_data(handle, slot: int) -> Tuple[int, int]:
+    """Device addresses (ints) of one slot's K and V."""
+    k = ctypes.c_void_p()
+    v = ctypes.c_void_p()
+    _check(lib().kv_cache_slot_data(handle, slot, ctypes.byref(k), ctypes.byref(v)))
+    return int(k.value), int(v.value)
+
+
+def kv_cache_destroy(handle) -> None:
+    lib().kv_cache_destroy(handle)
+
+
+def chunk_attention_fwd(handle, q, k_cur, v_cur, cur_frame_idx: Sequence[int], o, lse=None,
+                        softmax_scale: float = 0.0, stream=None) -> None:
+    _check(lib().chunk_attention_fwd(handle, _ptr(q), q.shape[0], _ptr(k_cur), _ptr(v_cur),
+                                     _i32(cur_frame_idx), len(cur_frame_idx),
+                                     float(softmax_scale), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def moba_attention_fwd(q, k, v, n_chunks: int, chunk_tokens: int, n_bidir_chunks: int, o,
+                       lse=None, softmax_scale: float = 0.0, stream=None) -> None:
+    lay = kvcr_moba_layout(n_chunks, chunk_tokens, n_bidir_chunks)
+    _check(lib().moba_attention_fwd(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(lay), q.shape[1],
+                                    q.shape[2], _dtype_code(q.dtype), float(softmax_scale),
+                                    _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def moba_classify_tiles(n_chunks: int, chunk_tokens: int, n_bidir_chunks: int, tile: int = 128):
+    import numpy as np
+    lay = kvcr_moba_layout(n_chunks, chunk_tokens, n_bidir_chunks)
+    L = (2 * n_chunks + n_bidir_chunks) * chunk_tokens
+    nt = (L + tile - 1) // tile
+    out = np.zeros((nt, nt), dtype=np.uint8)
+    _check(lib().moba_classify_tiles(ctypes.byref(lay), tile, out.ctypes.data, out.size))
+    return out
+
+
+def kvcr_check_status(stream=None) -> None:
+    _check(lib().kvcr_check_status(_stream(stream)))
+
+
+def kvcr_launch_count() -> int:
+    return int(lib().kvcr_launch_count())
+
+
+def kvcr_trace_enable(on: bool) -> None:
+    _check(lib().kvcr_trace_enable(int(bool(on))))
+
+
+def kvcr_trace_reset() -> None:
+    _check(lib().kvcr_trace_reset())
+
+
+def kvcr_trace_read(kernel_id: int) -> Tuple[int, float]:
+    n = ctypes.c_longlong()
+    ms = ctypes.c_double()
+    _check(lib().kvcr_trace_read(kernel_id, ctypes.byref(n), ctypes.byref(ms)))
+    return int(n.value), float(ms.value)
+
+
+# ------------------------------------------------------------- convenience ---
+
+class Cache:
+    """One layer's KV cache: owns the C handle and keeps its device storage alive."""
+
+    def __init__(self, sinks: int, window: int, tokens_per_frame: int, heads: int, head_dim: int,
+                 chunk_frames: int, rope=None, dtype="bf16", device="cuda",
+                 bookkeeping_only: bool = False):
+        self.sinks, self.window = sinks, window
+        self.T, self.H, self.D, self.F = tokens_per_frame, heads, head_dim, chunk_frames
+        self.rope = rope
+        self.dtype_code = _dtype_code(dtype)
+        self.storage = None
+        if not bookkeeping_only:
+            import torch
+            nbytes = kv_cache_storage_bytes(sinks, window, tokens_per_frame, heads, head_dim,
+                                            chunk_frames, rope is not None, self.dtype_code)
+            if nbytes == 0:
+                raise KvcrError(KVCR_ESHAPE, "invalid cache sizes")
+            self.storage = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.handle = kv_cache_init(sinks, window, tokens_per_frame, heads, head_dim,
+                                    chunk_frames, rope, self.dtype_code, self.storage)
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and _lib is not None:
+            kv_cache_destroy(h)
+            self.handle = None
+
+    @property
+    def torch_dtype(self):
+        import torch
+        return torch.bfloat16 if self.dtype_code == KVCR_BF16 else torch.float32
+
+    def append(self, k, v, frames: Sequence[int], stream=None) -> Tuple[List[int], List[int]]:
+        kv_cache_append_rope(self.handle, k, v, frames, stream)
+        return kv_cache_last_append(self.handle, len(frames))
+
+    def evict(self, keep_recent: int) -> List[int]:
+        return kv_cache_evict(self.handle, keep_recent)
+
+    def slot_map(self) -> List[int]:
+        return kv_cache_slot_map(self.handle, self.sinks + self.window)
+
+    def num_cached(self) -> int:
+        return kv_cache_num_cached(self.handle)
+
+    def slot_tensors(self, slot: int):
+        """Views (torch) of one slot's K and V, [T, H, D] in the cache dtype."""
+        import torch
+        kp, vp = kv_cache_slot_data(self.handle, slot)
+        esize = 2 if self.dtype_code == KVCR_BF16 else 4
+        n = self.T * self.H * self.D
+        base = self.storage.data_ptr()
+        flat = self.storage.view(self.torch_dtype) if self.storage.numel() % esize == 0 else None
+        k = flat[(kp - base) // esize:(kp - base) // esize + n].view(self.T, self.H, self.D)
+        v = flat[(vp - base) // esize:(vp - base) // esize + n].view(self.T, self.H, self.D)
+        return k, v
+
+    def attention(self, q, k_cur, v_cur, frames: Sequence[int], want_lse: bool = False,
+                  out=None, softmax_scale: float = 0.0, stream=None):
+        import torch
+        o = out if out is not None else torch.empty_like(q)
+        lse = None
+        if want_lse:
+            lse = torch.empty((self.H, q.shape[0]), dtype=torch.float32, device=q.device)
+        chunk_attention_fwd(self.handle, q, k_cur, v_cur, frames, o, lse, softmax_scale, stream)
+        return o, lse
+
+
+def default_scale(head_dim: int) -> float:
+    return 1.0 / math.sqrt(head_dim)

@@ -109,12 +109,15 @@ def classify_tiles_blocks(lay: MobaLayout, tile: int = 128) -> np.ndarray:
         # a representative position of each distinct chunk
         reps = [int(pos[np.nonzero((kind == a) & (idx == b))[0][0]]) for a, b in ids]
         spans.append(np.array(reps, dtype=np.int64))
+    # all key-side representatives in one array, with the tile each belongs to
+    krep = np.concatenate(spans)
+    starts = np.cumsum([0] + [len(sp) for sp in spans[:-1]])
     out = np.zeros((nt, nt), dtype=np.uint8)
     for i in range(nt):
-        qrep = spans[i]
-        for j in range(nt):
-            a = moba_allowed(qrep[:, None], spans[j][None, :], lay)
-            out[i, j] = TILE_FULL if a.all() else (TILE_PARTIAL if a.any() else TILE_EMPTY)
+        a = moba_allowed(spans[i][:, None], krep[None, :], lay)     # [rows reps, all key reps]
+        n_ok = np.add.reduceat(a.sum(axis=0), starts)                # allowed pairs per key tile
+        n_all = len(spans[i]) * np.diff(np.append(starts, krep.size))
+        out[i] = np.where(n_ok == n_all, TILE_FULL, np.where(n_ok > 0, TILE_PARTIAL, TILE_EMPTY))
     return out
 
 

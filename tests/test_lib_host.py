@@ -1,0 +1,157 @@
+"""CPU tests of the C-ABI library: it loads, exports every declared symbol, and its
+host bookkeeping / tile classification match the oracle bit-exactly.  No kernel
+runs here (bookkeeping-only caches; classification is host code)."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from kv_cache_chunk_ring_b200 import kvcr
+from kv_cache_chunk_ring_b200 import workloads as wl
+from oracle.cache import CacheModel
+from oracle.moba import MobaLayout, classify_tiles_blocks, classify_tiles_mask
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from kv_cache_chunk_ring_b200 import build
+    build.build()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "kvcr.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|void|size_t|long long|char)\s*\**\s*(\w+)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_bound_symbols():
+    assert sorted(kvcr.EXPORTS) == _declared()
+
+
+def test_library_exports_every_declared_symbol():
+    L = kvcr.lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def _bk_cache(S, W, T=4, H=1, D=64, F=4):
+    return kvcr.kv_cache_init(S, W, T, H, D, F, None, kvcr.KVCR_BF16, None)
+
+
+@pytest.mark.parametrize("spec", wl.ALL_ROLLOUTS, ids=lambda s: s.name)
+def test_bookkeeping_matches_oracle(spec):
+    sched = spec.window_schedule() if spec.window_seed is not None else None
+    cap = spec.window
+    h = _bk_cache(spec.sinks, cap, spec.tokens_per_frame, spec.heads, spec.head_dim,
+                  spec.chunk_frames)
+    ref = CacheModel(spec.sinks, cap)
+    try:
+        for c in range(spec.n_chunks):
+            if sched is not None:
+                ev_ref = ref.evict(sched[c])
+                assert kvcr.kv_cache_evict(h, sched[c]) == ev_ref
+            frames = spec.frames_of_chunk(c)
+            slots_ref, evicted_ref = ref.append(frames)
+            kvcr.kv_cache_append_rope(h, None, None, frames)
+            slots, evicted = kvcr.kv_cache_last_append(h, len(frames))
+            assert slots == slots_ref
+            assert evicted == evicted_ref
+            assert kvcr.kv_cache_slot_map(h, spec.sinks + cap) == ref.slot_map()
+            assert kvcr.kv_cache_num_cached(h) == ref.n_cached()
+    finally:
+        kvcr.kv_cache_destroy(h)
+
+
+def test_random_schedules_match_oracle():
+    rng = np.random.default_rng(21)
+    for trial in range(40):
+        S = int(rng.integers(0, 5))
+        W = int(rng.integers(0 if S > 0 else 1, 9))
+        F = int(rng.integers(1, 6))
+        h = _bk_cache(S, W, F=F)
+        ref = CacheModel(S, W)
+        f = int(rng.integers(0, 3))
+        for step in range(25):
+            if W > 0 and rng.random() < 0.3:
+                keep = int(rng.integers(0, W + 1))
+                assert kvcr.kv_cache_evict(h, keep) == ref.evict(keep)
+            n = int(rng.integers(0, F + 1))
+            frames = []
+            for _ in range(n):
+                f += int(rng.integers(1, 3))
+                frames.append(f)
+            if not frames:
+                continue
+            s_ref, e_ref = ref.append(frames)
+            kvcr.kv_cache_append_rope(h, None, None, frames)
+            assert kvcr.kv_cache_last_append(h, n) == (s_ref, e_ref)
+            assert kvcr.kv_cache_slot_map(h, S + W) == ref.slot_map()
+        kvcr.kv_cache_destroy(h)
+
+
+def test_errors_leave_state_unchanged():
+    h = _bk_cache(2, 2, F=2)
+    kvcr.kv_cache_append_rope(h, None, None, [0, 1])
+    before = kvcr.kv_cache_slot_map(h, 4)
+    with pytest.raises(kvcr.KvcrError) as e:
+        kvcr.kv_cache_append_rope(h, None, None, [1, 2])       # not increasing
+    assert e.value.code == kvcr.KVCR_ESTATE
+    with pytest.raises(kvcr.KvcrError) as e:
+        kvcr.kv_cache_append_rope(h, None, None, [5, 4])
+    assert e.value.code == kvcr.KVCR_ESTATE
+    assert kvcr.kv_cache_slot_map(h, 4) == before
+    with pytest.raises(kvcr.KvcrError) as e:
+        kvcr.kv_cache_evict(h, 3)
+    assert e.value.code == kvcr.KVCR_EINVAL
+    with pytest.raises(kvcr.KvcrError) as e:      # attention needs device storage
+        kvcr.lib()
+        rc = kvcr.lib().chunk_attention_fwd(h, None, 8, None, None, kvcr._i32([7]), 1, 0.0, None,
+                                            None, None)
+        kvcr._check(rc)
+    assert e.value.code == kvcr.KVCR_ESTATE
+    kvcr.kv_cache_destroy(h)
+
+
+def test_init_validation():
+    for args, code in [((0, 0), kvcr.KVCR_ESHAPE), ((20, 13), kvcr.KVCR_ESHAPE)]:
+        with pytest.raises(kvcr.KvcrError) as e:
+            _bk_cache(*args)
+        assert e.value.code == code
+    with pytest.raises(kvcr.KvcrError) as e:
+        kvcr.kv_cache_init(2, 2, 4, 1, 96, 2, None, kvcr.KVCR_BF16, None)
+    assert e.value.code == kvcr.KVCR_EUNSUPPORTED
+    bad = wl.RopeSpec(2, 3, 10, 10, 10)   # grid 2x3 != 4 tokens
+    with pytest.raises(kvcr.KvcrError) as e:
+        kvcr.kv_cache_init(2, 2, 4, 1, 64, 2, bad, kvcr.KVCR_BF16, None)
+    assert e.value.code == kvcr.KVCR_ESHAPE
+    assert kvcr.kv_cache_storage_bytes(0, 0, 4, 1, 64, 2, False, kvcr.KVCR_BF16) == 0
+
+
+def test_storage_bytes_cover_slots_and_scratch():
+    T, H, D, S, W, F = 1508, 12, 128, 6, 8, 4
+    frame = T * H * D * 2
+    n = kvcr.kv_cache_storage_bytes(S, W, T, H, D, F, True, kvcr.KVCR_BF16)
+    assert n >= 2 * (S + W) * frame + 2 * F * frame
+    assert n < 2 * (S + W) * frame + 2 * F * frame + 4 * T * D * 8 + 4096
+
+
+@pytest.mark.parametrize("n,c,m,tile", [(2, 5, 1, 4), (3, 7, 2, 4), (4, 3, 2, 8), (2, 16, 2, 16),
+                                        (3, 20, 1, 16), (5, 6, 3, 4), (2, 9, 0, 4), (3, 50, 2, 128),
+                                        (4, 200, 3, 128)])
+def test_classify_tiles_small_match_oracle(n, c, m, tile):
+    got = kvcr.moba_classify_tiles(n, c, m, tile)
+    ref = classify_tiles_mask(MobaLayout(n, c, m), tile)
+    assert np.array_equal(got, ref)
+
+
+def test_classify_tiles_full_size_matches_oracle():
+    spec = wl.MOBA_8x6032
+    got = kvcr.moba_classify_tiles(spec.n_chunks, spec.chunk_tokens, spec.n_bidir_chunks, 128)
+    ref = classify_tiles_blocks(MobaLayout(spec.n_chunks, spec.chunk_tokens, spec.n_bidir_chunks), 128)
+    assert got.shape == (1131, 1131)
+    assert np.array_equal(got, ref)
