@@ -372,7 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
 
     for (int j = 0; j < n_tiles; ++j) {
-      if (!(ok = wait_bar(&ctl->s_full[j & 1], (uint32_t)(j >> 1) & 1u, ctl))) break;
+      ok = wait_bar(&ctl->s_full[j & 1], (uint32_t)(j >> 1) & 1u, ctl);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {  // leave the loop warp-uniformly
+        ok = false;
+        break;
+      }
       tc_fence_after();
       __syncwarp();
       uint32_t s[128];
@@ -403,7 +407,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
       // PV of the previous tile must be done before P is overwritten or O rescaled.
       if (j >= 1) {
-        if (!(ok = wait_bar(&ctl->o_done, (uint32_t)(j - 1) & 1u, ctl))) break;
+        ok = wait_bar(&ctl->o_done, (uint32_t)(j - 1) & 1u, ctl);
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
       }
       const bool grow = m_new > m_ref + kRescaleLog2;
@@ -449,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
     // ---------------------------------------------------------- epilogue --
     if (ok && n_tiles > 0) ok = wait_bar(&ctl->o_done, (uint32_t)(n_tiles - 1) & 1u, ctl);
+    ok = __all_sync(0xFFFFFFFFu, ok);
     tc_fence_after();
     __syncwarp();
     const int row = q0 + r;
@@ -488,6 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

@@ -1,0 +1,82 @@
+"""Helpers shared by the GPU parity tests: device transfer, error metrics, and
+running a rollout through the C ABI in the same order as the oracle rollout."""
+from __future__ import annotations
+
+import math
+from typing import Callable, List, Optional
+
+import numpy as np
+
+# Tolerances on attention outputs against the fp64 oracle, per call:
+# max |O - O*| <= 2e-2 and ||O - O*||_2 / ||O*||_2 <= 5e-3 (bf16 inputs, fp32 accumulation).
+TOL_MAX_ABS = 2e-2
+TOL_REL_RMS = 5e-3
+# LSE is an fp32 log-sum-exp of bf16-rounded scores: an absolute bound.
+TOL_LSE = 2e-2
+
+
+def torch_dtype(dtype: str):
+    import torch
+    return torch.bfloat16 if dtype == "bf16" else torch.float32
+
+
+def to_dev(x: np.ndarray, dtype: str):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(
+        device="cuda", dtype=torch_dtype(dtype))
+
+
+def to_np(t) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def errors(got: np.ndarray, ref: np.ndarray):
+    d = got - ref
+    max_abs = float(np.abs(d).max()) if d.size else 0.0
+    nrm = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(d) / nrm) if nrm > 0 else float(np.linalg.norm(d))
+    return max_abs, rel
+
+
+def assert_close(got, ref, what: str = "", max_abs=TOL_MAX_ABS, rel_rms=TOL_REL_RMS):
+    ma, rr = errors(got, ref)
+    assert ma <= max_abs and rr <= rel_rms, f"{what}: max_abs={ma:.3e} rel_rms={rr:.3e}"
+    return ma, rr
+
+
+def rope_of(spec):
+    return spec.rope()
+
+
+def gpu_rollout(spec, chunks, rows_for: Optional[Callable] = None, use_rope: bool = True,
+                window_schedule: Optional[List[int]] = None):
+    """Run the rollout through the C ABI.  Returns dict of per-call outputs (rows
+    selected by rows_for, numpy fp64), LSEs, slot maps after each append, and the
+    Cache (for read-back)."""
+    import torch
+    from kv_cache_chunk_ring_b200.kvcr import Cache
+    cap = spec.window if window_schedule is None else max(spec.window, max(window_schedule))
+    cache = Cache(spec.sinks, cap, spec.tokens_per_frame, spec.heads, spec.head_dim,
+                  spec.chunk_frames, rope=spec.rope() if use_rope else None, dtype=spec.dtype)
+    out = dict(outputs=[], lses=[], slot_maps=[], appended=[], cache=cache)
+    for item in chunks:
+        c, s, frames = item["chunk"], item["step"], item["frames"]
+        if s == 0 and window_schedule is not None:
+            cache.evict(window_schedule[c])
+        q = to_dev(item["q"], spec.dtype)
+        k = to_dev(item["k"], spec.dtype)
+        v = to_dev(item["v"], spec.dtype)
+        o, lse = cache.attention(q, k, v, frames, want_lse=True)
+        rows = np.arange(q.shape[0]) if rows_for is None else np.asarray(rows_for(c, s))
+        idx = torch.from_numpy(rows).cuda()
+        out["outputs"].append(to_np(o.index_select(0, idx)))
+        out["lses"].append(lse.index_select(1, idx).cpu().numpy().astype(np.float64))
+        if s == spec.steps - 1:
+            out["appended"].append(cache.append(k, v, frames))
+            out["slot_maps"].append(cache.slot_map())
+    torch.cuda.synchronize()
+    return out
+
+
+def scale_of(spec) -> float:
+    return 1.0 / math.sqrt(spec.head_dim)
