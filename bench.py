@@ -1,0 +1,457 @@
+"""Benchmark: steady-state chunk step of the 832x464 single-layer rollout.
+
+One step = one 4-latent-frame chunk of the rollout at steady state: the chunk's
+queries attend 6 anchor + 8 window frames + the chunk itself (27144 keys,
+12 heads, head_dim 128, bf16) through ``chunk_attention_fwd`` (RoPE staging of
+Q and the current K, then tensor-core attention), then the chunk's K/V are
+appended to the cache through ``kv_cache_append_rope`` (RoPE of K, oldest
+non-anchor frames evicted).  The metric is useful attention TFLOP/s
+(4 * Lq * Lk * H * D per step), with ms/step, the attention kernel's share of
+the dense bf16 roofline and the append kernel's GB/s reported beside it.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
+layer cache (weak scaling, no collective on the data path); the timed region
+is bracketed by barriers and the max elapsed time over ranks is reported.
+``--impl reference`` times the CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from kv_cache_chunk_ring_b200 import workloads as wl  # noqa: E402
+
+SPEC = wl.VIDEO_832x464
+METRIC = "chunk-attention useful TFLOP/s & % of B200 bf16 peak; ms/chunk; append GB/s"
+UNIT = "TFLOP/s"
+STEADY_CHUNK = 4          # chunks 0-3 fill the cache; from chunk 4 on it holds 14 frames
+POOL = 3                  # distinct input chunks cycled through the timed steps
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def step_flops(spec=SPEC) -> float:
+    lq = spec.chunk_tokens
+    lk = (spec.sinks + spec.window + spec.chunk_frames) * spec.tokens_per_frame
+    return 4.0 * lq * lk * spec.heads * spec.head_dim
+
+
+def append_bytes(spec=SPEC) -> float:
+    # read K and V, write rotated K and V: 4 * F * T * H * D * 2 bytes
+    return 4.0 * spec.chunk_tokens * spec.heads * spec.head_dim * 2
+
+
+def config_dict(spec=SPEC) -> dict:
+    lk = (spec.sinks + spec.window + spec.chunk_frames) * spec.tokens_per_frame
+    return {
+        "workload": spec.name,
+        "heads": spec.heads, "head_dim": spec.head_dim,
+        "tokens_per_frame": spec.tokens_per_frame, "grid": [spec.grid_h, spec.grid_w],
+        "chunk_frames": spec.chunk_frames, "sinks": spec.sinks, "window": spec.window,
+        "q_tokens": spec.chunk_tokens, "keys": lk,
+        "step": "chunk_attention_fwd (RoPE stage + attention) + kv_cache_append_rope, steady state",
+        "l2": "inputs larger than L2: each step reads 130 MB of cached K/V + 55.6 MB chunk inputs",
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("attn_sm100.cu", "sm100_ptx.cuh", "kvcr_internal.h"):
+        with open(os.path.join(ROOT, "kv_cache_chunk_ring_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary,
+    or None when that summary is missing or was taken on different kernel source."""
+    p = os.path.join(ROOT, "profiles", "chunk_attn_832x464_ncu.md")
+    if not os.path.exists(p):
+        return None
+    src = None
+    traffic = None
+    for line in open(p):
+        if line.startswith("source-hash:"):
+            src = line.split(":", 1)[1].strip()
+        if line.startswith("dram-bytes-per-launch:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    if src != kernel_source_hash():
+        return None
+    return traffic
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        self.dev = ids[device_index] if device_index < len(ids) else str(device_index)
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            cols = [c.strip() for c in line.split(",")]
+            if len(cols) < 9:
+                continue
+            try:
+                sm.append(float(cols[1]))
+                mx = float(cols[2])
+            except ValueError:
+                continue
+            for n, c in zip(names, cols[5:9]):
+                if c.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- ours --
+
+def run_ours(args, rank: int, world: int, dist) -> dict:
+    import torch
+    from kv_cache_chunk_ring_b200 import build as _build
+    from kv_cache_chunk_ring_b200 import kvcr
+
+    if rank == 0 or not os.path.exists(os.path.join(ROOT, "kv_cache_chunk_ring_b200", "libkvcr.so")):
+        _build.build()
+    if dist is not None:
+        dist.barrier()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    spec = SPEC
+    T, H, D, F = spec.tokens_per_frame, spec.heads, spec.head_dim, spec.chunk_frames
+    stream = torch.cuda.current_stream()
+
+    cache = kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope())
+    # seeded synthetic chunks (each rank its own layer seed): fill chunks + a pool for timing
+    gen = wl.rollout_chunks(wl.shrink(spec, n_chunks=STEADY_CHUNK + POOL), layer=rank)
+    chunks = []
+    for item in gen:
+        chunks.append(tuple(torch.from_numpy(item[x]).to(dev, torch.bfloat16)
+                            for x in ("q", "k", "v")))
+    o = torch.empty_like(chunks[0][0])
+    frame = [0]
+
+    def step(i):
+        q, k, v = chunks[STEADY_CHUNK + (i % POOL)] if i >= 0 else chunks[i + STEADY_CHUNK]
+        frames = list(range(frame[0], frame[0] + F))
+        cache.attention(q, k, v, frames, out=o)
+        cache.append(k, v, frames)
+        frame[0] += F
+
+    # fill the cache to steady state (chunks 0-3), then warm up
+    for i in range(-STEADY_CHUNK, 0):
+        step(i)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert cache.num_cached() == spec.sinks + spec.window
+
+    # ---------------- timed region (device events, no tracing) ----------------
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = kvcr.kvcr_launch_count()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    launches = kvcr.kvcr_launch_count() - launches0
+    clocks = sampler.stop()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # ---------------- per-kernel times (traced pass, same steps) ----------------
+    kvcr.kvcr_trace_reset()
+    kvcr.kvcr_trace_enable(True)
+    for i in range(args.steps):
+        step(i)
+    torch.cuda.synchronize()
+    kvcr.kvcr_trace_enable(False)
+    kt = {}
+    for kid, name in kvcr.KERNEL_NAMES.items():
+        n, ms = kvcr.kvcr_trace_read(kid)
+        if n:
+            kt[name] = {"launches": n, "avg_ms": ms / n}
+    kvcr.kvcr_trace_reset()
+
+    # ---------------- end to end through the public API with host buffers ----------------
+    host = [tuple(t.cpu().pin_memory() for t in chunks[STEADY_CHUNK + j]) for j in range(POOL)]
+    dq = torch.empty_like(chunks[0][0])
+    dk = torch.empty_like(chunks[0][1])
+    dvv = torch.empty_like(chunks[0][2])
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+
+    def e2e_step(i):
+        hq, hk, hv = host[i % POOL]
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dvv.copy_(hv, non_blocking=True)
+        frames = list(range(frame[0], frame[0] + F))
+        cache.attention(dq, dk, dvv, frames, out=o)
+        cache.append(dk, dvv, frames)
+        frame[0] += F
+        o_host.copy_(o, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    kvcr.kvcr_check_status()
+
+    flops = step_flops(spec)
+    value = world * args.steps * flops / (elapsed_ms * 1e-3) / 1e12
+    e2e_value = world * args.steps * flops / (e2e_ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    attn = kt.get("chunk_attn", {})
+    attn_ms = attn.get("avg_ms", float("nan"))
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    app = kt.get("append_rope", {})
+    app_gbs = append_bytes(spec) / (app.get("avg_ms", float("nan")) * 1e-3) / 1e9
+    chunk_bytes = spec.chunk_tokens * H * D * 2
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(spec),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": recorded_traffic(),
+                     "kernel": "chunk_attn (tcgen05 attention, one launch per step)",
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)"},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
+                "h2d_bytes_per_step": 3 * chunk_bytes, "d2h_bytes_per_step": chunk_bytes,
+                "ms_per_step": round(e2e_ms / args.steps, 4)},
+        "gpu_launches": int(launches),
+        "kernels": {k: {"launches": v["launches"], "avg_ms": round(v["avg_ms"], 5)}
+                    for k, v in kt.items()},
+        "attn_ms_per_call": round(attn_ms + kt.get("rope_stage", {}).get("avg_ms", 0.0), 5),
+        "attn_kernel_pct_of_peak": round(100 * achieved / peak, 2),
+        "append_gb_s": round(app_gbs, 1),
+        "append_hbm_frac": round(app_gbs / float(peaks["hbm_gbs"]), 4),
+        "clocks": clocks,
+    }
+    return out
+
+
+# ---------------------------------------------------------------- oracle ----
+
+def oracle_sample(rows: int, seed_chunk=STEADY_CHUNK):
+    """Build a bounded oracle sample of one steady-state chunk step and return a
+    callable that runs it plus the useful FLOPs it covers."""
+    from oracle.rollout import rollout  # noqa: F401  (oracle package)
+    from oracle.attn import attention
+    from oracle.rope import rope3d, rope_positions
+
+    spec = wl.shrink(SPEC, n_chunks=seed_chunk + 1)
+    items = list(wl.rollout_chunks(spec))
+    pairs = (spec.rope().pairs_t, spec.rope().pairs_h, spec.rope().pairs_w)
+    T = spec.tokens_per_frame
+    # the steady-state cache content: anchors 0-5 and window frames 8-15 (rotated K, V)
+    cached_k, cached_v = [], []
+    keep = list(range(spec.sinks)) + list(range(seed_chunk * spec.chunk_frames - spec.window,
+                                               seed_chunk * spec.chunk_frames))
+    for it in items[:-1]:
+        t, h, w = rope_positions(it["frames"], spec.grid_h, spec.grid_w)
+        kr = rope3d(it["k"], t, h, w, pairs)
+        for n, f in enumerate(it["frames"]):
+            if f in keep:
+                cached_k.append(kr[n * T:(n + 1) * T])
+                cached_v.append(it["v"][n * T:(n + 1) * T].astype(np.float64))
+    cur = items[-1]
+    sel = wl.sample_rows(spec.chunk_tokens, rows, 2024)
+    lk = (len(keep) + spec.chunk_frames) * T
+    flops = 4.0 * len(sel) * lk * spec.heads * spec.head_dim
+    scale = 1.0 / math.sqrt(spec.head_dim)
+
+    def run():
+        t, h, w = rope_positions(cur["frames"], spec.grid_h, spec.grid_w)
+        qr = rope3d(cur["q"][sel], t[sel], h[sel], w[sel], pairs)
+        kc = rope3d(cur["k"], t, h, w, pairs)
+        k_all = np.concatenate(cached_k + [kc])
+        v_all = np.concatenate(cached_v + [cur["v"].astype(np.float64)])
+        return attention(qr, k_all, v_all, scale)
+
+    return run, flops, len(sel)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s: float = 12.0) -> dict:
+    run, flops, n = oracle_sample(32)
+    t0 = time.perf_counter()
+    run()
+    t1 = time.perf_counter() - t0
+    per_row = t1 / n
+    rows = int(max(32, min(2048, budget_s / max(per_row, 1e-6))))
+    run, flops, n = oracle_sample(rows)
+    t0 = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"one steady-state chunk step of {SPEC.name} restricted to {n} of "
+                      f"{SPEC.chunk_tokens} query rows (all 12 heads, RoPE of the rows' Q and "
+                      f"the chunk's K, attention over 27144 keys), numpy fp64; "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args) -> dict:
+    """The oracle as the reference arm: each step = the bounded oracle sample."""
+    per_step_budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    run, flops, n = oracle_sample(32)
+    t0 = time.perf_counter()
+    run()
+    per_row = (time.perf_counter() - t0) / n
+    rows = int(max(16, min(2048, per_step_budget / max(per_row, 1e-6))))
+    run, flops, n = oracle_sample(rows)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    value = args.steps * flops / dt / 1e12
+    sample = (f"per step: one steady-state chunk step of {SPEC.name} restricted to {n} query rows"
+              f" (all heads, 27144 keys), numpy fp64 on host cores")
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(), "impl": "reference",
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)))
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        out = run_ours(args, rank, world, dist)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(out))
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
