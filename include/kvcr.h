@@ -168,6 +168,29 @@ int chunk_attention_fwd(kvcr_cache *c, const void *q, int n_q, const void *k_cur
                         const void *v_cur, const int32_t *cur_frame_idx, int n_cur_frames,
                         float softmax_scale, void *o, float *lse, void *stream);
 
+/* chunk_attention_fwd() for callers that cannot allocate device memory at the
+ * time of the call -- for example code that runs while a stream is being
+ * captured into a CUDA graph, real-time loops that cannot afford the implicit
+ * synchronisation of cudaMalloc/cudaFree, or hosts whose memory pool gives the
+ * library exactly the cache buffer.  (The pages describe no such call; it is a
+ * property of this library.)  Arguments, result and errors are those of
+ * chunk_attention_fwd().  The difference: the rotated queries and current-chunk
+ * keys are staged in a fixed 36 MiB array that the library holds in device
+ * memory on every GPU where it is loaded (until the process exits), not in the
+ * cache's scratch region.  A chunk whose staging needs more than that
+ * (2 x n_cur_frames * tokens_per_frame * heads * head_dim * sizeof(dtype), each
+ * half rounded up to 256 bytes) is rejected with KVCR_ESHAPE before anything is
+ * launched; a bf16 chunk of 4 frames x 1508 tokens x 12 heads x 128 fits.  The
+ * call allocates nothing.  The first call on a device looks up the array's
+ * address once for that device; make that first call before any stream capture.
+ * All calls on a device share the array, which keeps the last call's contents
+ * (nothing in it needs to start at zero); calls whose GPU work overlaps -- on
+ * different streams or from different host threads -- race on it. */
+int chunk_attention_fwd_static_scratch(kvcr_cache *c, const void *q, int n_q,
+                                       const void *k_cur, const void *v_cur,
+                                       const int32_t *cur_frame_idx, int n_cur_frames,
+                                       float softmax_scale, void *o, float *lse, void *stream);
+
 /* Attention under the MoBA mask over one sequence of L = layout tokens.
  * q, k, v, o: device [L][heads][head_dim] bf16 (head_dim 128 or 64); lse nullable
  * fp32 [heads][L].  128 x 128 tiles of the score matrix with no allowed entry

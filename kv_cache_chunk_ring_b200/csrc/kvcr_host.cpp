@@ -30,6 +30,7 @@
 
 #include "kvcr_internal.h"
 #include "moba_layout.h"
+#include "static_scratch.h"
 
 using namespace kvcr;
 
@@ -639,6 +640,139 @@ int chunk_attention_fwd(kvcr_cache* c, const void* q, int n_q, const void* k_cur
       e = launch_attn_f32(p, s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd: fp32 attention launch");
+  }
+  return KVCR_OK;
+}
+
+// ============================================= chunk attention, static scratch
+// Same computation as chunk_attention_fwd(); the rotated queries and current
+// keys are staged in the library's fixed device array instead of the cache's
+// scratch region, so the call needs no memory beyond its inputs, outputs and
+// the cache.  The first call on a device looks the array's address up (once
+// per device); make that first call before any stream capture.
+int chunk_attention_fwd_static_scratch(kvcr_cache* c, const void* q, int n_q, const void* k_cur,
+                                       const void* v_cur, const int32_t* cur_frame_idx,
+                                       int n_cur_frames, float softmax_scale, void* o, float* lse,
+                                       void* stream) {
+  const char* fn = "chunk_attention_fwd_static_scratch";
+  if (c == nullptr) return fail(KVCR_EINVAL, std::string(fn) + ": cache is NULL");
+  if (!c->has_storage) return fail(KVCR_ESTATE, std::string(fn) + ": bookkeeping-only cache");
+  if (n_cur_frames < 1 || n_cur_frames > c->F)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_cur_frames must be in [1, chunk_frames]");
+  if (n_q < 0) return fail(KVCR_ESHAPE, std::string(fn) + ": n_q < 0");
+  const int n_cur = n_cur_frames * c->T;
+  if (c->rope && n_q != n_cur)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": with RoPE n_q must be n_cur_frames * T");
+  int rc = check_frames(c, cur_frame_idx, n_cur_frames, fn);
+  if (rc) return rc;
+  if (n_q == 0) return KVCR_OK;
+  if (!q || !k_cur || !v_cur || !o) return fail(KVCR_EINVAL, std::string(fn) + ": NULL tensor");
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(o))
+    return fail(KVCR_EINVAL, std::string(fn) + ": tensors must be 16-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(KVCR_EINVAL, std::string(fn) + ": lse must be 4-byte aligned");
+  if ((long long)n_q * c->H * c->D > (1LL << 31) - 1)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_q too large");
+  // staging needs: rotated Q then rotated current K, each 256-byte aligned
+  const size_t half = align_up((size_t)n_cur * c->H * c->D * c->esize, 256);
+  if (c->rope && 2 * half > kStaticScratchBytes)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": the chunk needs " + std::to_string(2 * half) +
+                                 " bytes of staging, more than the fixed " +
+                                 std::to_string(kStaticScratchBytes) + "-byte array");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)c->D);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  int slots[kMaxSlots];
+  int n_vis = 0;
+  for (int i = 0; i < c->S + c->W; ++i)
+    if (c->slot_frame[i] >= 0) slots[n_vis++] = i;
+
+  const void* q_src = q;
+  const void* k_src = k_cur;
+  if (c->rope) {
+    void* scratch = nullptr;
+    cudaError_t e = static_scratch_address(&scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd_static_scratch: array address");
+    uint8_t* qs = static_cast<uint8_t*>(scratch);
+    uint8_t* ks = qs + half;
+    RopeCopyParams p;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(c, p);
+    p.src_a = q;
+    p.src_b = k_cur;
+    p.dst_a = qs;
+    p.dst_b = ks;
+    p.rotate_a = 1;
+    p.rotate_b = 1;
+    p.n_frames = n_cur_frames;
+    const long long frame_elems = (long long)c->T * c->H * c->D;
+    for (int f = 0; f < n_cur_frames; ++f) {
+      p.dst_frame_off[f] = f * frame_elems;
+      p.src_frame[f] = f;
+    }
+    fill_ttab(c, p, cur_frame_idx, n_cur_frames);
+    {
+      LaunchScope scope(KVCR_K_ROPE_STAGE, s);
+      e = launch_rope_copy(p, c->dtype, s, c->n_sm);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd_static_scratch: stage launch");
+    q_src = qs;
+    k_src = ks;
+  }
+
+  if (c->dtype == KVCR_BF16) {
+    ChunkAttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t dq[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_q};
+    const uint64_t dn[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_cur};
+    rc = encode_bf16_map(&p.tm_q, q_src, 3, dq);
+    if (!rc) rc = encode_bf16_map(&p.tm_kn, k_src, 3, dn);
+    if (!rc) rc = encode_bf16_map(&p.tm_vn, v_cur, 3, dn);
+    if (rc) return rc;
+    p.tm_kc = c->tm_kc;
+    p.tm_vc = c->tm_vc;
+    p.c.o = o;
+    p.c.lse = lse;
+    p.c.n_q = n_q;
+    p.c.H = c->H;
+    p.c.scale_log2 = (float)(scale * 1.4426950408889634);
+    p.s.T = c->T;
+    p.s.n_vis = n_vis;
+    p.s.tiles_per_slot = (c->T + kTile - 1) / kTile;
+    p.s.n_cur = n_cur;
+    p.s.cur_tiles = (n_cur + kTile - 1) / kTile;
+    for (int i = 0; i < n_vis; ++i) p.s.slots[i] = slots[i];
+    cudaError_t e;
+    {
+      LaunchScope scope(KVCR_K_CHUNK_ATTN, s);
+      e = launch_chunk_attn_sm100(p, c->D, (n_q + kTile - 1) / kTile, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd_static_scratch: attention launch");
+  } else {
+    F32AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = static_cast<const float*>(q_src);
+    p.kc = reinterpret_cast<const float*>(c->storage + c->lay.k_off);
+    p.vc = reinterpret_cast<const float*>(c->storage + c->lay.v_off);
+    p.kn = static_cast<const float*>(k_src);
+    p.vn = static_cast<const float*>(v_cur);
+    p.o = static_cast<float*>(o);
+    p.lse = lse;
+    p.n_q = n_q;
+    p.H = c->H;
+    p.D = c->D;
+    p.T = c->T;
+    p.n_vis = n_vis;
+    p.n_cur = n_cur;
+    p.scale = scale;
+    for (int i = 0; i < n_vis; ++i) p.slots[i] = slots[i];
+    cudaError_t e;
+    {
+      LaunchScope scope(KVCR_K_ATTN_F32, s);
+      e = launch_attn_f32(p, s);
+    }
+    if (e != cudaSuccess)
+      return cuda_fail(e, "chunk_attention_fwd_static_scratch: fp32 attention launch");
   }
   return KVCR_OK;
 }

@@ -32,7 +32,7 @@ EXPORTS = [
     "kv_cache_storage_bytes", "kv_cache_init", "kv_cache_append_rope", "kv_cache_evict",
     "kv_cache_slot_map", "kv_cache_last_append", "kv_cache_num_cached", "kv_cache_slot_data",
     "kv_cache_destroy",
-    "chunk_attention_fwd", "moba_attention_fwd", "moba_classify_tiles", "kvcr_check_status",
+    "chunk_attention_fwd", "chunk_attention_fwd_static_scratch", "moba_attention_fwd", "moba_classify_tiles", "kvcr_check_status",
     "kvcr_last_error", "kvcr_launch_count", "kvcr_trace_enable", "kvcr_trace_reset",
     "kvcr_trace_read",
 ]
@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
         "kv_cache_destroy": (None, [c_p]),
         "chunk_attention_fwd": (c_int, [c_p, c_p, c_int, c_p, c_p, i32p, c_int, c_f, c_p, c_p,
                                         c_p]),
+        "chunk_attention_fwd_static_scratch": (c_int, [c_p, c_p, c_int, c_p, c_p, i32p, c_int,
+                                                       c_f, c_p, c_p, c_p]),
         "moba_attention_fwd": (c_int, [c_p, c_p, c_p, ctypes.POINTER(kvcr_moba_layout), c_int,
                                        c_int, c_int, c_f, c_p, c_p, c_p]),
         "moba_classify_tiles": (c_int, [ctypes.POINTER(kvcr_moba_layout), c_int, c_p, c_sz]),
@@ -204,6 +206,15 @@ def chunk_attention_fwd(handle, q, k_cur, v_cur, cur_frame_idx: Sequence[int], o
     _check(lib().chunk_attention_fwd(handle, _ptr(q), q.shape[0], _ptr(k_cur), _ptr(v_cur),
                                      _i32(cur_frame_idx), len(cur_frame_idx),
                                      float(softmax_scale), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def chunk_attention_fwd_static_scratch(handle, q, k_cur, v_cur, cur_frame_idx: Sequence[int], o,
+                                       lse=None, softmax_scale: float = 0.0,
+                                       stream=None) -> None:
+    """chunk_attention_fwd staged in the library's fixed device array (allocates nothing)."""
+    _check(lib().chunk_attention_fwd_static_scratch(
+        handle, _ptr(q), q.shape[0], _ptr(k_cur), _ptr(v_cur), _i32(cur_frame_idx),
+        len(cur_frame_idx), float(softmax_scale), _ptr(o), _ptr(lse), _stream(stream)))
 
 
 def moba_attention_fwd(q, k, v, n_chunks: int, chunk_tokens: int, n_bidir_chunks: int, o,
