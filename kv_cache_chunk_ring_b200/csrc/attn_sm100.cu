@@ -11,24 +11,31 @@
 // teacher-forcing + bidirectional rule ("Infinite Worlds with Versatile
 // Interactions", causal-pretraining paragraph) and skips empty 128 x 128 tiles.
 //
-// Design (one CTA = one 128-query tile of one head, 192 threads):
-//   warp 4      TMA producer: Q once, then K and V tiles (128 keys x D) through
-//               a 2-stage ring; cached-frame tiles come from a 4D tensor map
-//               (D, H, T, slot) so a tile never crosses a slot and the frame's
-//               ragged tail is zero-filled.
-//   warp 5      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
-//               S buffers (128 columns fp32 each), O += P_j V_j into TMEM O.
-//               UMMA 128 x 128 x 16 (S) and 128 x D x 16 (PV), bf16 in, fp32 out.
-//   warps 0-3   softmax: thread r owns query row r = TMEM lane r, so the row
-//               max / sum are in-thread; exp2 with the scale folded in; P is
-//               written bf16 into a 128B-swizzled shared tile (the UMMA A
-//               operand); the running max is only moved (and O rescaled in
-//               TMEM) when it grows by more than 2^8, and the final
-//               normalisation uses the same stale max, so the result is exact.
-//   epilogue    O / l -> bf16 -> global, LSE = (m + log2 l) ln 2.
-// Every wait is bounded: after 2 s a thread records KVCR_ETIMEOUT in the
-// device status word, raises the CTA abort flag and the CTA drains its
-// in-flight copies and MMAs before freeing TMEM and returning.
+// Design (one CTA = two 128-query tiles of one head, 384 threads = 3 warpgroups;
+// the producer warpgroup gives registers to the two softmax warpgroups):
+//   warp 8      TMA producer: Q0 and Q1 once, then K and V tiles (128 keys x D)
+//               through a 2-stage ring shared by both query tiles; cached-frame
+//               tiles come from a 4D tensor map (D, H, T, slot) so a tile never
+//               crosses a slot and the frame's ragged tail is zero-filled.
+//   warp 9      MMA issuer (one thread), tcgen05.mma kind::f16, fp32 in TMEM:
+//                 S_t = Q_t K_j^T          (A, B from shared memory)
+//                 O_t += P_t V_j           (A = P_t from TMEM, B = V from smem)
+//               issued in the order  PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so the
+//               tensor core works on one tile while the other tile's softmax
+//               runs.  P_t overwrites S_t in TMEM (bf16 pairs packed in 32-bit
+//               columns); MMAs of one thread execute in issue order, so S_t(j+1)
+//               is written only after PV_t(j) has read P_t(j).
+//   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r owns
+//               query row r = TMEM lane r, so the row max / sum stay in-thread;
+//               exp2 with the scale folded in, a quarter of it evaluated on the
+//               FMA pipe (range reduction + cubic) to offload the SFU; the
+//               running max only moves (and O_t is rescaled in TMEM) when it
+//               grows by more than 2^8, and the final normalisation uses the same
+//               stale max, so the result is exact.
+//   epilogue    each softmax warpgroup: O_t / l -> bf16 -> global, LSE.
+// Every wait is bounded: after 2 s a thread records KVCR_ETIMEOUT in the device
+// status word, raises the CTA abort flag and the CTA drains its in-flight
+// copies and MMAs before freeing TMEM and returning.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -44,25 +51,30 @@ namespace {
 using namespace ptx;
 
 constexpr int kStages = 2;
-constexpr int kThreads = 192;
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
+constexpr int kThreads = 384;
+// Register budgets after setmaxnreg: launch 384 x 168; producer warpgroup
+// (TMA warp, MMA warp, two idle warps) 80, softmax warpgroups 208 each:
+// 128 x (208 + 208 + 80) = 63488 <= 384 x 168 = 64512.
+constexpr uint32_t kRegsProducer = 80;
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;  // O accumulator columns [256, 256 + D)
+// TMEM columns: S_t / P_t at t * 128, O_t at 256 + t * 128.
+constexpr uint32_t kTmemS = 0;
+constexpr uint32_t kTmemO = 256;
 
 struct __align__(8) Ctl {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t p_full;
-  uint64_t o_done;
+  uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
   int n_tiles;
   int pad;
-  uint16_t tiles[kMobaMaxTiles];  // MoBA: key tile | class << 12
+  uint16_t tiles[kMobaMaxTiles];  // MoBA: key tile | class(tile 0) << 12 | class(tile 1) << 14
 };
 
 template <int HD>
@@ -70,12 +82,10 @@ struct Smem {
   static constexpr int kBoxes = HD / 64;          // 64-element (128-byte) boxes per row
   static constexpr int kBoxBytes = 128 * 128;     // 128 rows x 128 bytes
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kPBytes = 2 * kBoxBytes;   // 128 x 128 bf16
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kQ = 0;                    // Q0, Q1
+  static constexpr int kK = kQ + 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kP = kV + kStages * kTileBytes;
-  static constexpr int kCtl = kP + kPBytes;
+  static constexpr int kCtl = kV + kStages * kTileBytes;
   static constexpr int kBytes = kCtl + (int)sizeof(Ctl) + 1024;  // + 1024 B alignment slack
 };
 
@@ -84,7 +94,8 @@ struct TileRef {
   int slot;   // cache slot (map 0, chunk attention)
   int row0;   // first key row of the tile within its tensor
   int valid;  // keys of the tile inside the tensor
-  int cls;    // kTileFull / kTilePartial
+  int cls0;   // class for query tile 0 / 1 (kTileFull: no mask needed)
+  int cls1;
 };
 
 __device__ __forceinline__ TileRef tile_ref(const ChunkAttnParams& p, const Ctl*, int j) {
@@ -104,7 +115,7 @@ __device__ __forceinline__ TileRef tile_ref(const ChunkAttnParams& p, const Ctl*
     t.row0 = tt * kTile;
     t.valid = min(kTile, p.s.n_cur - t.row0);
   }
-  t.cls = kTileFull;
+  t.cls0 = t.cls1 = kTileFull;
   return t;
 }
 
@@ -115,7 +126,8 @@ __device__ __forceinline__ TileRef tile_ref(const MobaAttnParams& p, const Ctl* 
   t.slot = 0;
   t.row0 = (int)(e & 0xFFFu) * kTile;
   t.valid = min(kTile, p.s.L - t.row0);
-  t.cls = (int)(e >> 12);
+  t.cls0 = (int)((e >> 12) & 3u);
+  t.cls1 = (int)((e >> 14) & 3u);
   return t;
 }
 
@@ -175,21 +187,29 @@ __device__ __forceinline__ void prefetch_maps(const MobaAttnParams& p) {
   prefetch_tmap(&p.tm_v);
 }
 
-// MoBA: list the non-empty key tiles of query tile qt (one warp).
-__device__ void build_moba_list(const MobaAttnParams& p, int qt, Ctl* ctl, int lane) {
+// MoBA: list the key tiles that are non-empty for query tile 2u or 2u + 1
+// (one warp), with each tile's class for both query tiles.
+__device__ void build_moba_list(const MobaAttnParams& p, int unit, Ctl* ctl, int lane) {
   const MobaLay lay{p.s.n_chunks, p.s.chunk_tokens, p.s.n_bidir, p.s.L};
-  const int r0 = qt * kTile;
-  const int r1 = min(r0 + kTile, p.s.L);
+  const int qt0 = 2 * unit;
+  const int r0 = qt0 * kTile;
+  const int r1 = min(r0 + 2 * kTile, p.s.L);
   int lo, hi;
   moba_row_bounds(lay, r0, r1, lo, hi);
   const int kt0 = lo / kTile, kt1 = (hi + kTile - 1) / kTile;
   int count = 0;
   for (int base = kt0; base < kt1; base += 32) {
     const int kt = base + lane;
-    const int cls = kt < kt1 ? moba_classify(lay, qt, kt, kTile) : (int)kTileEmpty;
-    const unsigned ball = __ballot_sync(0xFFFFFFFFu, cls != kTileEmpty);
-    if (cls != kTileEmpty)
-      ctl->tiles[count + __popc(ball & ((1u << lane) - 1u))] = (uint16_t)(kt | (cls << 12));
+    int c0 = kTileEmpty, c1 = kTileEmpty;
+    if (kt < kt1) {
+      c0 = moba_classify(lay, qt0, kt, kTile);
+      c1 = moba_classify(lay, qt0 + 1, kt, kTile);
+    }
+    const bool keep = c0 != kTileEmpty || c1 != kTileEmpty;
+    const unsigned ball = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep)
+      ctl->tiles[count + __popc(ball & ((1u << lane) - 1u))] =
+          (uint16_t)(kt | (c0 << 12) | (c1 << 14));
     count += __popc(ball);
   }
   if (lane == 0) ctl->n_tiles = count;
@@ -205,10 +225,27 @@ __device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
 }
 
 // 2^x on the SFU (MUFU.EX2); -inf -> +0.
-__device__ __forceinline__ float ex2(float x) {
+__device__ __forceinline__ float ex2_sfu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA / integer pipes (keeps the SFU free).  Cody-Waite style range
+// reduction x = n + f, n = round(x) taken from the low mantissa bits of
+// x + 1.5 * 2^23, f in [-1/2, 1/2]; 2^f by the cubic 1 + f (c1 + f (c2 + f c3))
+// fitted here to 2^f on [-1/2, 1/2] for least maximum relative error
+// (Lawson-weighted least squares; max relative error 1.02e-4, below the bf16
+// rounding of P).  n is added to the exponent field.  x is clamped at -127,
+// where the result is exactly +0 (p(0) = 1), so masked scores give 0.
+__device__ __forceinline__ float ex2_fma(float x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c1 = 0.6932829022f, c2 = 0.2422103733f, c3 = 0.0550085828f;
+  x = fmaxf(x, -127.0f);
+  const float t = x + kShift;
+  const float f = x - (t - kShift);
+  const float p = fmaf(f, fmaf(f, fmaf(f, c3, c2), c1), 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -224,15 +261,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  int qt, h;
+  int unit, h;  // unit = pair of query tiles (rows [256 unit, 256 unit + 256))
   if constexpr (kMoba) {
     h = blockIdx.x / p.s.n_row_tiles;
-    qt = p.s.order[blockIdx.x - h * p.s.n_row_tiles];
+    unit = p.s.order[blockIdx.x - h * p.s.n_row_tiles];
   } else {
-    qt = blockIdx.x;
+    unit = blockIdx.x;
     h = blockIdx.y;
   }
-  const int q0 = qt * kTile;
+  const int q0 = unit * 2 * kTile;
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
@@ -242,10 +279,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       mbar_init(&ctl->v_full[s], 1);
       mbar_init(&ctl->v_empty[s], 1);
     }
-    mbar_init(&ctl->s_full[0], 1);
-    mbar_init(&ctl->s_full[1], 1);
-    mbar_init(&ctl->p_full, 128);
-    mbar_init(&ctl->o_done, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctl->s_full[t], 1);
+      mbar_init(&ctl->p_full[t], 128);
+      mbar_init(&ctl->o_done[t], 1);
+    }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     if constexpr (!kMoba) ctl->n_tiles = p.s.n_vis * p.s.tiles_per_slot + p.s.cur_tiles;
@@ -256,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     tmem_relinquish();
   }
   if constexpr (kMoba) {
-    if (warp == kWarpTma) build_moba_list(p, qt, ctl, lane);
+    if (warp == kWarpTma) build_moba_list(p, unit, ctl, lane);
   }
   tc_fence_before();
   __syncthreads();
@@ -264,14 +302,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const uint32_t tmem = ctl->tmem_base;
   const int n_tiles = ctl->n_tiles;
 
+  if (warp >= 8) {
+  setmaxnreg_dec<kRegsProducer>();
   if (warp == kWarpTma) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0 && n_tiles > 0) {
       prefetch_maps(p);
-      mbar_arrive_expect_tx(&ctl->q_full, L::kTileBytes);
+      mbar_arrive_expect_tx(&ctl->q_full, 2 * L::kTileBytes);
 #pragma unroll
-      for (int b = 0; b < L::kBoxes; ++b)
-        tma_load_3d(smem + L::kQ + b * L::kBoxBytes, &p.tm_q, &ctl->q_full, b * 64, h, q0);
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int b = 0; b < L::kBoxes; ++b)
+          tma_load_3d(smem + L::kQ + t * L::kTileBytes + b * L::kBoxBytes, &p.tm_q, &ctl->q_full,
+                      b * 64, h, q0 + t * kTile);
       int issued = 0;  // tiles whose K and V loads were issued
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
@@ -282,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         mbar_arrive_expect_tx(&ctl->k_full[st], L::kTileBytes);
         load_kv_tile<HD>(p, t, false, smem + L::kK + st * L::kTileBytes, &ctl->k_full[st], h);
         if (!(ok = wait_bar(&ctl->v_empty[st], ph ^ 1u, ctl))) {
-          issued = j;  // K of tile j in flight: drained below with the V side skipped
+          issued = j;
           drain_wait(&ctl->k_full[st], ph);
           break;
         }
@@ -309,41 +352,66 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const uint32_t sQ = smem_u32(smem + L::kQ);
       const uint32_t sK = smem_u32(smem + L::kK);
       const uint32_t sV = smem_u32(smem + L::kV);
-      const uint32_t sP = smem_u32(smem + L::kP);
-      bool ok = wait_bar(&ctl->q_full, 0, ctl);
-      tc_fence_after();
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          const int st = j % kStages;
-          if (!(ok = wait_bar(&ctl->k_full[st], (uint32_t)(j / kStages) & 1u, ctl))) break;
-          tc_fence_after();
-          const uint32_t d = tmem + (uint32_t)(j & 1) * 128u;
-          const uint32_t kb = sK + st * L::kTileBytes;
+      // S_t(j) = Q_t K_j^T
+      auto issue_s = [&](int t, int j) {
+        const uint32_t d = tmem + kTmemS + (uint32_t)t * 128u;
+        const uint32_t qb = sQ + t * L::kTileBytes;
+        const uint32_t kb = sK + (j % kStages) * L::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-            umma_ss(d, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescS,
-                    kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&ctl->s_full[j & 1]);
-          umma_commit(&ctl->k_empty[st]);
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+          umma_ss(d, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescS,
+                  kk > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int st = jj % kStages;
-          if (!(ok = wait_bar(&ctl->p_full, (uint32_t)jj & 1u, ctl))) break;
-          if (!(ok = wait_bar(&ctl->v_full[st], (uint32_t)(jj / kStages) & 1u, ctl))) break;
-          tc_fence_after();
-          const uint32_t vb = sV + st * L::kTileBytes;
+      };
+      // O_t += P_t(j) V_j, P_t in TMEM (8 packed columns per 16 keys)
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t pa = tmem + kTmemS + (uint32_t)t * 128u;
+        const uint32_t d = tmem + kTmemO + (uint32_t)t * 128u;
+        const uint32_t vb = sV + (j % kStages) * L::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {
-            const uint32_t poff = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-            umma_ss(tmem + kTmemO, sdesc_sw128(sP + poff, 16, 1024),
-                    sdesc_sw128(vb + kk * 16 * 128, L::kBoxBytes, 1024), kIdescO,
-                    (jj > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&ctl->o_done);
-          umma_commit(&ctl->v_empty[st]);
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ts(d, pa + kk * 8, sdesc_sw128(vb + kk * 16 * 128, L::kBoxBytes, 1024), kIdescO,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait_bar(&ctl->q_full, 0, ctl) && wait_bar(&ctl->k_full[0], 0, ctl);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        umma_commit(&ctl->s_full[0]);
+        issue_s(1, 0);
+        umma_commit(&ctl->s_full[1]);
+        umma_commit(&ctl->k_empty[0]);
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int st = j % kStages;
+        const bool more = j + 1 < n_tiles;
+        // tile 0: PV_0(j), then S_0(j+1)
+        if (!(ok = wait_bar(&ctl->p_full[0], (uint32_t)j & 1u, ctl))) break;
+        if (!(ok = wait_bar(&ctl->v_full[st], (uint32_t)(j / kStages) & 1u, ctl))) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          if (!(ok = wait_bar(&ctl->k_full[(j + 1) % kStages],
+                              (uint32_t)((j + 1) / kStages) & 1u, ctl)))
+            break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+          umma_commit(&ctl->s_full[0]);
+        } else {
+          umma_commit(&ctl->o_done[0]);
+        }
+        // tile 1: PV_1(j), then S_1(j+1)
+        if (!(ok = wait_bar(&ctl->p_full[1], (uint32_t)j & 1u, ctl))) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(&ctl->v_empty[st]);
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit(&ctl->s_full[1]);
+          umma_commit(&ctl->k_empty[(j + 1) % kStages]);
+        } else {
+          umma_commit(&ctl->o_done[1]);
         }
       }
       if (!ok) {
@@ -351,12 +419,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         drain_wait(&ctl->drain, 0);
       }
     }
+  }
   } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // --------------------------------------------- softmax + epilogue ----
-    const int r = threadIdx.x;                      // query row in the tile = TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int tq = warp >> 2;                        // query tile of this warpgroup
+    const int r = threadIdx.x & 127;                 // row in the tile = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + kTmemS + (uint32_t)tq * 128u;
+    const uint32_t o_addr = tmem + lane_base + kTmemO + (uint32_t)tq * 128u;
     const float sl2 = p.c.scale_log2;
-    uint8_t* sP = smem + L::kP;
+    const int row_g = q0 + tq * kTile + r;           // global query row
     float m_ref = -INFINITY;                        // running (possibly stale) max, log2 units
     float l_sum = 0.f;
     bool ok = true;
@@ -365,110 +438,108 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     int a0 = 0, b0 = 0, a1 = 0, b1 = 0;
     if constexpr (kMoba) {
       const MobaLay lay{p.s.n_chunks, p.s.chunk_tokens, p.s.n_bidir, p.s.L};
-      const int row = min(q0 + r, p.s.L - 1);
+      const int row = min(row_g, p.s.L - 1);
       int lo[2] = {0, 0}, hi[2] = {0, 0};
       moba_row_intervals(lay, row, row + 1, lo, hi, 2);
       a0 = lo[0]; b0 = hi[0]; a1 = lo[1]; b1 = hi[1];
     }
 
     for (int j = 0; j < n_tiles; ++j) {
-      ok = wait_bar(&ctl->s_full[j & 1], (uint32_t)(j >> 1) & 1u, ctl);
+      ok = wait_bar(&ctl->s_full[tq], (uint32_t)j & 1u, ctl);
       if (!__all_sync(0xFFFFFFFFu, ok)) {  // leave the loop warp-uniformly
         ok = false;
         break;
       }
       tc_fence_after();
-      __syncwarp();
       uint32_t s[128];
-      const uint32_t sbase = tmem + lane_base + (uint32_t)(j & 1) * 128u;
-      tmem_ld_32x32b_x32(sbase + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld_32x32b_x32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld_32x32b_x32(sbase + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld_32x32b_x32(sbase + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_ld_32x32b_x32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld_32x32b_x32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld_32x32b_x32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld_32x32b_x32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_ld_wait();
 
       const TileRef t = tile_ref(p, ctl, j);
-      if (t.valid < kTile || (kMoba && t.cls == kTilePartial)) {
+      const int cls = tq == 0 ? t.cls0 : t.cls1;
+      if (t.valid < kTile || (kMoba && cls != kTileFull)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int base = t.row0 + 32 * c;
           uint32_t keep = bit_range(0, t.valid - 32 * c);
-          if (kMoba && t.cls == kTilePartial)
+          if (kMoba && cls != kTileFull)
             keep &= bit_range(a0 - base, b0 - base) | bit_range(a1 - base, b1 - base);
 #pragma unroll
           for (int n = 0; n < 32; ++n)
             if (!((keep >> n) & 1u)) s[32 * c + n] = __float_as_uint(-INFINITY);
         }
       }
-      float mx = -INFINITY;
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int n = 0; n < 128; ++n) mx = fmaxf(mx, __uint_as_float(s[n]));
-      const float m_new = fmaxf(m_ref, mx * sl2);
-
-      // PV of the previous tile must be done before P is overwritten or O rescaled.
-      if (j >= 1) {
-        ok = wait_bar(&ctl->o_done, (uint32_t)(j - 1) & 1u, ctl);
-        if (!__all_sync(0xFFFFFFFFu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      for (int n = 0; n < 128; n += 2) {
+        mx0 = fmaxf(mx0, __uint_as_float(s[n]));
+        mx1 = fmaxf(mx1, __uint_as_float(s[n + 1]));
       }
+      const float m_new = fmaxf(m_ref, fmaxf(mx0, mx1) * sl2);
+
+      // O_t is stable here: S_t(j) was committed after PV_t(j-1).
       const bool grow = m_new > m_ref + kRescaleLog2;
       if (__any_sync(0xFFFFFFFFu, grow)) {
-        const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+        const float alpha = (m_ref == -INFINITY) ? 0.f : ex2_sfu(m_ref - m_new);
         if (j >= 1) {
-          __syncwarp();
 #pragma unroll 1
           for (int c = 0; c < HD / 32; ++c) {
             uint32_t o[32];
-            const uint32_t oaddr = tmem + lane_base + kTmemO + c * 32;
-            tmem_ld_32x32b_x32(oaddr, o);
+            tmem_ld_32x32b_x32(o_addr + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int n = 0; n < 32; ++n) o[n] = __float_as_uint(__uint_as_float(o[n]) * alpha);
-            tmem_st_32x32b_x32(oaddr, o);
+            tmem_st_32x32b_x32(o_addr + c * 32, o);
           }
-          tmem_st_wait();
         }
         l_sum *= alpha;
         if (m_new != -INFINITY) m_ref = m_new;
       }
       const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
+      float l0 = 0.f, l1 = 0.f;
 #pragma unroll
-      for (int g = 0; g < 16; ++g) {                // 16 groups of 8 keys
-        uint32_t packed[4];
+      for (int c = 0; c < 4; ++c) {                 // 4 groups of 32 keys -> 16 packed columns
+        uint32_t packed[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[g * 8 + 2 * e]), sl2, -msub));
-          const float p1 = ex2(fmaf(__uint_as_float(s[g * 8 + 2 * e + 1]), sl2, -msub));
-          l_sum += p0 + p1;
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = fmaf(__uint_as_float(s[32 * c + 2 * e]), sl2, -msub);
+          const float x1 = fmaf(__uint_as_float(s[32 * c + 2 * e + 1]), sl2, -msub);
+          float p0, p1;
+          if (e >= 12) {                             // a quarter of the exps on the FMA pipe
+            p0 = ex2_fma(x0);
+            p1 = ex2_fma(x1);
+          } else {
+            p0 = ex2_sfu(x0);
+            p1 = ex2_sfu(x1);
+          }
+          l0 += p0;
+          l1 += p1;
           __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
           packed[e] = *reinterpret_cast<uint32_t*>(&b2);
         }
-        const int box = g >> 3, c16 = g & 7;
-        uint8_t* dst = sP + box * L::kBoxBytes + r * 128 + ((c16 ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        tmem_st_32x32b_x16(s_addr + c * 16, packed);
       }
-      fence_proxy_async_smem();
+      l_sum += l0 + l1;
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&ctl->p_full);
+      mbar_arrive(&ctl->p_full[tq]);
     }
 
     // ---------------------------------------------------------- epilogue --
-    if (ok && n_tiles > 0) ok = wait_bar(&ctl->o_done, (uint32_t)(n_tiles - 1) & 1u, ctl);
+    if (ok && n_tiles > 0) ok = wait_bar(&ctl->o_done[tq], 0, ctl);
     ok = __all_sync(0xFFFFFFFFu, ok);
     tc_fence_after();
-    __syncwarp();
-    const int row = q0 + r;
-    const bool row_ok = ok && row < p.c.n_q;
+    const bool row_ok = ok && row_g < p.c.n_q;
     const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.c.o) + ((size_t)row * p.c.H + h) * HD;
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.c.o) + ((size_t)row_g * p.c.H + h) * HD;
 #pragma unroll 1
     for (int c = 0; c < HD / 32; ++c) {
       uint32_t o[32];
       if (n_tiles > 0 && ok) {
-        tmem_ld_32x32b_x32(tmem + lane_base + kTmemO + c * 32, o);
+        tmem_ld_32x32b_x32(o_addr + c * 32, o);
         tmem_ld_wait();
       } else {
 #pragma unroll
@@ -490,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     if (row_ok && p.c.lse != nullptr) {
       const float lse = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
-      p.c.lse[(size_t)h * p.c.n_q + row] = lse;
+      p.c.lse[(size_t)h * p.c.n_q + row_g] = lse;
     }
   }
 
@@ -521,7 +592,7 @@ cudaError_t launch_impl(const Params& p, dim3 grid, cudaStream_t s) {
 
 cudaError_t launch_chunk_attn_sm100(const ChunkAttnParams& p, int head_dim, int n_q_tiles,
                                     cudaStream_t s) {
-  dim3 grid((unsigned)n_q_tiles, (unsigned)p.c.H);
+  dim3 grid((unsigned)((n_q_tiles + 1) / 2), (unsigned)p.c.H);
   if (head_dim == 128) return launch_impl<128, false>(p, grid, s);
   if (head_dim == 64) return launch_impl<64, false>(p, grid, s);
   return cudaErrorInvalidValue;

@@ -805,16 +805,19 @@ int moba_classify_tiles(const kvcr_moba_layout* layout, int tile, uint8_t* cls, 
 }
 
 namespace {
-// Non-empty key tiles of each 128-row tile (tiles hit by the union of the
-// rows' allowed key intervals), and the row tiles ordered heaviest first.
+// Work units are pairs of 128-row query tiles (one CTA each).  A unit's work
+// is the number of key tiles hit by the union of its rows' allowed key
+// intervals; units are ordered heaviest first.
 void moba_order(const MobaLay& l, std::vector<uint16_t>& order) {
-  const int nt = (l.L + kTile - 1) / kTile;
+  constexpr int kUnitRows = 2 * kTile;
+  const int nt = (l.L + kUnitRows - 1) / kUnitRows;
   std::vector<int> work(nt);
   std::vector<std::pair<int, int>> iv;
-  int lo[2 * kTile + 8], hi[2 * kTile + 8];
+  constexpr int kCap = 2 * kUnitRows + 8;
+  int lo[kCap], hi[kCap];
   for (int i = 0; i < nt; ++i) {
-    const int r0 = i * kTile, r1 = std::min(r0 + kTile, l.L);
-    const int n = moba_row_intervals(l, r0, r1, lo, hi, 2 * kTile + 8);
+    const int r0 = i * kUnitRows, r1 = std::min(r0 + kUnitRows, l.L);
+    const int n = moba_row_intervals(l, r0, r1, lo, hi, kCap);
     iv.clear();
     for (int k = 0; k < n; ++k)
       if (hi[k] > lo[k]) iv.push_back({lo[k] / kTile, (hi[k] - 1) / kTile});
@@ -892,7 +895,7 @@ int moba_attention_fwd(const void* q, const void* k, const void* v,
   p->s.chunk_tokens = l.c;
   p->s.n_bidir = l.m;
   p->s.L = l.L;
-  p->s.n_row_tiles = (l.L + kTile - 1) / kTile;
+  p->s.n_row_tiles = (l.L + 2 * kTile - 1) / (2 * kTile);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   {

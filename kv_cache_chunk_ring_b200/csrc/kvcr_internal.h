@@ -52,8 +52,8 @@ struct ChunkSched {
 struct MobaSched {
   int n_chunks, chunk_tokens, n_bidir;
   int L;
-  int n_row_tiles;
-  uint16_t order[kMobaMaxTiles];  // row tiles, heaviest first
+  int n_row_tiles;                    // work units per head: pairs of 128-row query tiles
+  uint16_t order[kMobaMaxTiles / 2];  // units, heaviest first
 };
 
 struct AttnCommon {
