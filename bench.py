@@ -414,6 +414,163 @@ def run_reference(args) -> dict:
     }
 
 
+# ------------------------------------------------------- other workloads ----
+# Single-GPU timings of the other workloads; inputs are seeded N(0,1) bf16 drawn on the
+# device with torch (same distribution as the parity inputs, generated faster).
+
+def _randn(shape, gen):
+    import torch
+    return torch.randn(shape, generator=gen, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+
+
+def _timed(fn, steps, warmup):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_layers30(args) -> dict:
+    """30 layers x 4 denoising steps per chunk (120 attention calls + 30 appends)."""
+    import torch
+    from kv_cache_chunk_ring_b200 import build as _build
+    from kv_cache_chunk_ring_b200 import kvcr
+    _build.build()
+    spec = wl.VIDEO_832x464_30L
+    T, H, D, F = spec.tokens_per_frame, spec.heads, spec.head_dim, spec.chunk_frames
+    caches = [kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope())
+              for _ in range(spec.layers)]
+    gen = torch.Generator(device="cuda").manual_seed(spec.seed)
+    pool = [tuple(_randn((spec.chunk_tokens, H, D), gen) for _ in range(3)) for _ in range(6)]
+    o = torch.empty_like(pool[0][0])
+    frame = [0]
+    n_call = [0]
+
+    def chunk():
+        frames = list(range(frame[0], frame[0] + F))
+        for li, c in enumerate(caches):
+            for s in range(spec.steps):
+                q, k, v = pool[n_call[0] % len(pool)]
+                n_call[0] += 1
+                c.attention(q, k, v, frames, out=o)
+            c.append(k, v, frames)
+        frame[0] += F
+
+    for _ in range(STEADY_CHUNK):
+        chunk()
+    kvcr.kvcr_trace_reset()
+    ms = _timed(chunk, args.steps, args.warmup)
+    kvcr.kvcr_trace_enable(True)
+    chunk()
+    torch.cuda.synchronize()
+    kvcr.kvcr_trace_enable(False)
+    kt = {name: kvcr.kvcr_trace_read(kid) for kid, name in kvcr.KERNEL_NAMES.items()}
+    kvcr.kvcr_trace_reset()
+    flops = spec.layers * spec.steps * step_flops(spec)
+    app_n, app_ms = kt["append_rope"]
+    return {"workload": spec.name, "ms_per_chunk": round(ms, 3),
+            "attention_tflops_per_chunk": round(flops / 1e12, 2),
+            "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": UNIT,
+            "attn_kernel_ms": round(kt["chunk_attn"][1] / max(1, kt["chunk_attn"][0]), 4),
+            "append_kernel_us": round(1e3 * app_ms / max(1, app_n), 2),
+            "append_gb_s": round(append_bytes(spec) / (app_ms / max(1, app_n) * 1e-3) / 1e9, 1),
+            "steps": args.steps, "warmup": args.warmup,
+            "note": "steady-state chunks (cache full); 30 independent layer caches, 5.0 GB"}
+
+
+def moba_useful_flops(spec) -> float:
+    n, m, c = spec.n_chunks, spec.n_bidir_chunks, spec.chunk_tokens
+    pairs = (n * (n + 1) // 2 + n * (n - 1) // 2 + n + m * m) * c * c
+    return 4.0 * pairs * spec.heads * spec.head_dim
+
+
+def run_moba(args) -> dict:
+    import torch
+    from kv_cache_chunk_ring_b200 import build as _build
+    from kv_cache_chunk_ring_b200 import kvcr
+    _build.build()
+    spec = wl.MOBA_8x6032
+    gen = torch.Generator(device="cuda").manual_seed(spec.seed)
+    shape = (spec.seq_len, spec.heads, spec.head_dim)
+    q, k, v = (_randn(shape, gen) for _ in range(3))
+    o = torch.empty_like(q)
+
+    def call():
+        kvcr.moba_attention_fwd(q, k, v, spec.n_chunks, spec.chunk_tokens, spec.n_bidir_chunks, o)
+
+    ms = _timed(call, args.steps, args.warmup)
+    kvcr.kvcr_check_status()
+    flops = moba_useful_flops(spec)
+    peaks, kind = load_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": spec.name, "ms_per_call": round(ms, 3), "useful_tflop": round(flops / 1e12, 3),
+            "value": round(tf, 2), "unit": UNIT, "frac_of_peak": round(tf / peaks["bf16_tflops"], 4),
+            "steps": args.steps, "warmup": args.warmup}
+
+
+def run_dynwin(args) -> dict:
+    """720p rollout, 6 anchors, window drawn per chunk from U{2..8}, plus cross-attention."""
+    import torch
+    from kv_cache_chunk_ring_b200 import build as _build
+    from kv_cache_chunk_ring_b200 import kvcr
+    _build.build()
+    spec = wl.VIDEO_720P_DYN
+    T, H, D, F = spec.tokens_per_frame, spec.heads, spec.head_dim, spec.chunk_frames
+    sched = spec.window_schedule()
+    self_c = kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope())
+    cross_c = kvcr.Cache(1, 0, spec.text_env, H, D, 1, rope=None)
+    gen = torch.Generator(device="cuda").manual_seed(spec.seed)
+    pool = [tuple(_randn((spec.chunk_tokens, H, D), gen) for _ in range(3)) for _ in range(3)]
+    env_k, env_v = _randn((spec.text_env, H, D), gen), _randn((spec.text_env, H, D), gen)
+    loc = [(_randn((spec.text_local, H, D), gen), _randn((spec.text_local, H, D), gen))
+           for _ in range(3)]
+    cross_c.append(env_k, env_v, [0])
+    o = torch.empty_like(pool[0][0])
+    ox = torch.empty_like(pool[0][0])
+    state = {"c": 0, "flops": 0.0}
+
+    def chunk():
+        c = state["c"]
+        w = sched[c % len(sched)]
+        self_c.evict(w)
+        frames = list(range(c * F, (c + 1) * F))
+        q, k, v = pool[c % 3]
+        lk = (self_c.num_cached() + F) * T
+        self_c.attention(q, k, v, frames, out=o)
+        lq, lv = loc[c % 3]
+        cross_c.attention(q, lq, lv, [c + 1], out=ox)
+        self_c.append(k, v, frames)
+        state["flops"] += 4.0 * spec.chunk_tokens * (lk + spec.text_env + spec.text_local) * H * D
+        state["c"] = c + 1
+
+    for _ in range(STEADY_CHUNK):
+        chunk()
+    for _ in range(args.warmup):
+        chunk()
+    torch.cuda.synchronize()
+    state["flops"] = 0.0
+    n = max(args.steps, len(sched) - state["c"])
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        chunk()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    return {"workload": spec.name, "ms_per_chunk": round(ms, 3), "chunks_timed": n,
+            "value": round(state["flops"] / n / (ms * 1e-3) / 1e12, 2), "unit": UNIT,
+            "note": "per chunk: evict(W_t), self-attention, cross-attention (512 text keys), append"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -421,6 +578,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="chunk", choices=["chunk", "layers30", "moba", "dynwin"],
+                    help="chunk: the 832x464 steady-state step (the bench line); the others "
+                         "print single-GPU timings of the other workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -430,6 +590,11 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)))
+        return
+    if args.workload != "chunk":
+        fn = {"layers30": run_layers30, "moba": run_moba, "dynwin": run_dynwin}[args.workload]
+        if rank == 0:
+            print(json.dumps(fn(args)))
         return
 
     dist = None

@@ -14,10 +14,10 @@
 // 2 tensors x (read + write) x T x H x D x sizeof(elem); the angle tables are
 // a few KB and stay in L1/L2.
 //
-// Layout: one thread owns one 16-byte vector of a and the matching vector of
-// b (8 bf16 = 4 pairs, or 4 fp32 = 2 pairs), so loads and stores are
-// coalesced 16-byte accesses; a grid-stride loop over (frame, token, head,
-// vector) keeps the grid at a multiple of the SM count.
+// Layout: a warp moves one token (all heads) at a time with coalesced 16-byte
+// loads and stores, several vectors in flight per lane; a lane's vectors all
+// cover the same rotary pairs, so their (cos, sin) are fetched once per token.
+// The grid is one wave of resident CTAs (a multiple of the SM count).
 #include <cuda_bf16.h>
 
 #include "kvcr_internal.h"
@@ -39,15 +39,6 @@ __device__ __forceinline__ void st_vec(void* p, uint4 v) {
                : "memory");
 }
 
-// (cos, sin) of pair i for a token at (frame slot fr, row hh, col ww)
-__device__ __forceinline__ float2 angle_cs(const RopeCopyParams& p, int fr, int hh, int ww, int i) {
-  if (i < p.pairs_t) return p.ttab[fr][i];
-  i -= p.pairs_t;
-  if (i < p.pairs_h) return p.htab[hh * p.pairs_h + i];
-  i -= p.pairs_h;
-  return p.wtab[ww * p.pairs_w + i];
-}
-
 __device__ __forceinline__ void rot(float& x0, float& x1, float2 cs) {
   const float y0 = x0 * cs.x - x1 * cs.y;
   const float y1 = x0 * cs.y + x1 * cs.x;
@@ -55,85 +46,137 @@ __device__ __forceinline__ void rot(float& x0, float& x1, float2 cs) {
   x1 = y1;
 }
 
-__device__ __forceinline__ uint4 rotate_bf16x8(uint4 v, const RopeCopyParams& p, int fr, int hh,
-                                               int ww, int pair0) {
+template <int kPairs>
+__device__ __forceinline__ uint4 rotate_vec(uint4 v, const float2 (&cs)[4]);
+
+// 8 bf16 = 4 pairs
+template <>
+__device__ __forceinline__ uint4 rotate_vec<4>(uint4 v, const float2 (&cs)[4]) {
   uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     __nv_bfloat162 b2 = *reinterpret_cast<__nv_bfloat162*>(&w[k]);
     float2 f = __bfloat1622float2(b2);
-    rot(f.x, f.y, angle_cs(p, fr, hh, ww, pair0 + k));
+    rot(f.x, f.y, cs[k]);
     b2 = __floats2bfloat162_rn(f.x, f.y);
     w[k] = *reinterpret_cast<uint32_t*>(&b2);
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ __forceinline__ uint4 rotate_f32x4(uint4 v, const RopeCopyParams& p, int fr, int hh,
-                                              int ww, int pair0) {
+// 4 fp32 = 2 pairs
+template <>
+__device__ __forceinline__ uint4 rotate_vec<2>(uint4 v, const float2 (&cs)[4]) {
   float f[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
                 __uint_as_float(v.w)};
-  rot(f[0], f[1], angle_cs(p, fr, hh, ww, pair0));
-  rot(f[2], f[3], angle_cs(p, fr, hh, ww, pair0 + 1));
+  rot(f[0], f[1], cs[0]);
+  rot(f[2], f[3], cs[1]);
   return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
                     __float_as_uint(f[3]));
 }
 
+// One warp moves one token (H x D elements of a and of b) at a time.  A token
+// is H * D / kPerVec 16-byte vectors; lane l takes vectors l, l + 32, ..., and
+// because D / kPerVec divides 32, every vector of a lane covers the same
+// kPairsPerVec rotary pairs: the lane fetches their (cos, sin) once per token
+// (t-axis pairs once per frame) and reuses them for every head.
 template <typename Elem, int D>
 __global__ void __launch_bounds__(256) rope_copy_kernel(const __grid_constant__ RopeCopyParams p) {
   constexpr int kPerVec = 16 / sizeof(Elem);          // elements per 16-byte vector
   constexpr int kPairsPerVec = kPerVec / 2;
   constexpr int kVecPerRow = D / kPerVec;             // vectors per (token, head)
+  constexpr int kBatch = 6;                           // vectors in flight per lane and tensor
   const int f = blockIdx.y;                           // destination frame
-  const unsigned vec_per_frame = (unsigned)p.T * p.H * kVecPerRow;
-  const long long in_base = (long long)p.src_frame[f] * p.T * p.H * D;
-  const long long out_base = p.dst_frame_off[f];
-  const Elem* src_a = static_cast<const Elem*>(p.src_a) + in_base;
-  const Elem* src_b = static_cast<const Elem*>(p.src_b) + in_base;
-  Elem* dst_a = static_cast<Elem*>(p.dst_a) + out_base;
-  Elem* dst_b = static_cast<Elem*>(p.dst_b) + out_base;
-  for (unsigned r = blockIdx.x * blockDim.x + threadIdx.x; r < vec_per_frame;
-       r += gridDim.x * blockDim.x) {
-    const unsigned row = r / kVecPerRow;              // token * H + head
-    const int vi = (int)(r - row * kVecPerRow);
-    const int tok = (int)(row / (unsigned)p.H);
-    const int hh = tok / p.grid_w;
-    const int ww = tok - hh * p.grid_w;
-    const int pair0 = vi * kPairsPerVec;
-    uint4 a = ld_stream(src_a + (size_t)r * kPerVec);
-    uint4 b = ld_stream(src_b + (size_t)r * kPerVec);
-    if constexpr (sizeof(Elem) == 2) {
-      if (p.rotate_a) a = rotate_bf16x8(a, p, f, hh, ww, pair0);
-      if (p.rotate_b) b = rotate_bf16x8(b, p, f, hh, ww, pair0);
-    } else {
-      if (p.rotate_a) a = rotate_f32x4(a, p, f, hh, ww, pair0);
-      if (p.rotate_b) b = rotate_f32x4(b, p, f, hh, ww, pair0);
+  const int lane = threadIdx.x & 31;
+  const int vpt = p.H * kVecPerRow;                   // vectors per token
+  const int n_mine = (vpt - lane + 31) / 32;          // vectors of this lane per token
+  const int pair0 = (lane % kVecPerRow) * kPairsPerVec;
+  const long long tok_elems = (long long)p.H * D;
+  const Elem* src_a = static_cast<const Elem*>(p.src_a) + (long long)p.src_frame[f] * p.T * tok_elems;
+  const Elem* src_b = static_cast<const Elem*>(p.src_b) + (long long)p.src_frame[f] * p.T * tok_elems;
+  Elem* dst_a = static_cast<Elem*>(p.dst_a) + p.dst_frame_off[f];
+  Elem* dst_b = static_cast<Elem*>(p.dst_b) + p.dst_frame_off[f];
+
+  // axis and index of this lane's pairs; t-axis (cos, sin) are per frame
+  int axis[4], jx[4];
+  float2 cs_t[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    int i = pair0 + k;
+    axis[k] = i < p.pairs_t ? 0 : (i < p.pairs_t + p.pairs_h ? 1 : 2);
+    jx[k] = axis[k] == 0 ? i : (axis[k] == 1 ? i - p.pairs_t : i - p.pairs_t - p.pairs_h);
+    cs_t[k] = (k < kPairsPerVec && axis[k] == 0 && (p.rotate_a || p.rotate_b))
+                  ? p.ttab[f][jx[k] < kMaxPairsT ? jx[k] : 0]
+                  : make_float2(1.f, 0.f);
+  }
+  const int warps_total = gridDim.x * (blockDim.x / 32);
+  for (int tok = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); tok < p.T;
+       tok += warps_total) {
+    float2 cs[4];
+    if (p.rotate_a || p.rotate_b) {
+      const int hh = tok / p.grid_w;
+      const int ww = tok - hh * p.grid_w;
+#pragma unroll
+      for (int k = 0; k < kPairsPerVec; ++k) {
+        if (axis[k] == 0) cs[k] = cs_t[k];
+        else if (axis[k] == 1) cs[k] = p.htab[hh * p.pairs_h + jx[k]];
+        else cs[k] = p.wtab[ww * p.pairs_w + jx[k]];
+      }
     }
-    st_vec(dst_a + (size_t)r * kPerVec, a);
-    st_vec(dst_b + (size_t)r * kPerVec, b);
+    const long long base = (long long)tok * tok_elems;
+    for (int k0 = 0; k0 < n_mine; k0 += kBatch) {
+      uint4 a[kBatch], b[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        if (k0 + k < n_mine) {
+          const long long off = base + (long long)(lane + 32 * (k0 + k)) * kPerVec;
+          a[k] = ld_stream(src_a + off);
+          b[k] = ld_stream(src_b + off);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        if (k0 + k < n_mine) {
+          const long long off = base + (long long)(lane + 32 * (k0 + k)) * kPerVec;
+          uint4 ra = a[k], rb = b[k];
+          if (p.rotate_a) ra = rotate_vec<kPairsPerVec>(ra, cs);
+          if (p.rotate_b) rb = rotate_vec<kPairsPerVec>(rb, cs);
+          st_vec(dst_a + off, ra);
+          st_vec(dst_b + off, rb);
+        }
+      }
+    }
   }
 }
 
 }  // namespace
 
-cudaError_t launch_rope_copy(const RopeCopyParams& p, kvcr_dtype dtype, cudaStream_t s, int n_sm) {
-  if (p.n_frames <= 0) return cudaSuccess;
-  const int per_vec = dtype == KVCR_BF16 ? 8 : 4;
-  const long long per_frame = (long long)p.T * p.H * (p.D / per_vec);
-  if (per_frame == 0) return cudaSuccess;
-  // About 8 resident 256-thread CTAs per SM in total, split over the frames.
-  long long want = (per_frame + 255) / 256;
-  long long gx = ((long long)n_sm * 8 + p.n_frames - 1) / p.n_frames;
-  if (want < gx) gx = want;
-  dim3 grid((unsigned)gx, (unsigned)p.n_frames);
-  if (dtype == KVCR_BF16) {
-    if (p.D == 128) rope_copy_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
-    else rope_copy_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
-  } else {
-    if (p.D == 128) rope_copy_kernel<float, 128><<<grid, 256, 0, s>>>(p);
-    else rope_copy_kernel<float, 64><<<grid, 256, 0, s>>>(p);
+namespace {
+template <typename Elem, int D>
+cudaError_t launch_one(const RopeCopyParams& p, cudaStream_t s, int n_sm) {
+  static int per_sm = 0;  // resident CTAs per SM, from the occupancy calculator
+  if (per_sm == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rope_copy_kernel<Elem, D>,
+                                                                  256, 0);
+    if (e != cudaSuccess || per_sm < 1) per_sm = 1;
   }
+  // One wave: every resident CTA slot busy, split evenly over the frames; each
+  // of a CTA's 8 warps takes one token at a time.
+  const long long want = (p.T + 7) / 8;
+  long long gx = ((long long)n_sm * per_sm + p.n_frames - 1) / p.n_frames;
+  if (want < gx) gx = want;
+  if (gx < 1) gx = 1;
+  rope_copy_kernel<Elem, D><<<dim3((unsigned)gx, (unsigned)p.n_frames), 256, 0, s>>>(p);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_rope_copy(const RopeCopyParams& p, kvcr_dtype dtype, cudaStream_t s, int n_sm) {
+  if (p.n_frames <= 0 || p.T <= 0) return cudaSuccess;
+  if (dtype == KVCR_BF16)
+    return p.D == 128 ? launch_one<__nv_bfloat16, 128>(p, s, n_sm)
+                      : launch_one<__nv_bfloat16, 64>(p, s, n_sm);
+  return p.D == 128 ? launch_one<float, 128>(p, s, n_sm) : launch_one<float, 64>(p, s, n_sm);
 }
 
 }  // namespace kvcr
