@@ -27,8 +27,8 @@
 //               is written only after PV_t(j) has read P_t(j).
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r owns
 //               query row r = TMEM lane r, so the row max / sum stay in-thread;
-//               exp2 with the scale folded in, a quarter of it evaluated on the
-//               FMA pipe (range reduction + cubic) to offload the SFU; the
+//               exp2 with the scale folded in, part of it evaluated on the FMA
+//               pipe (range reduction + cubic, packed fp32x2) to offload the SFU; the
 //               running max only moves (and O_t is rescaled in TMEM) when it
 //               grows by more than 2^8, and the final normalisation uses the same
 //               stale max, so the result is exact.
@@ -60,6 +60,9 @@ constexpr uint32_t kRegsSoftmax = 208;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr float kRescaleLog2 = 8.0f;
+// Of the 16 key pairs in each 32-key group, pairs [0, kExpSfuPairs) take exp2 on
+// the SFU and the rest on the FMA pipe.
+constexpr int kExpSfuPairs = 12;
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S_t / P_t at t * 128, O_t at 256 + t * 128.
 constexpr uint32_t kTmemS = 0;
@@ -140,6 +143,25 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Ctl* ct
       atomicExch(&g_attn_status, (int)KVCR_ETIMEOUT);
       *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
       return false;
+    }
+  }
+  return true;
+}
+
+// Same contract as wait_bar, for the single MMA-issuing thread: it polls with the
+// non-suspending test so it reacts to a completed phase without a sleep quantum.
+__device__ __forceinline__ bool spin_bar(uint64_t* bar, uint32_t parity, Ctl* ctl) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  uint32_t n = 0;
+  while (!mbar_test_wait(bar, parity)) {
+    if ((++n & 255u) == 0u) {
+      if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
+      if (globaltimer() - t0 > (uint64_t)kWaitTimeoutNs) {
+        atomicExch(&g_attn_status, (int)KVCR_ETIMEOUT);
+        *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+        return false;
+      }
     }
   }
   return true;
@@ -231,21 +253,30 @@ __device__ __forceinline__ float ex2_sfu(float x) {
   return y;
 }
 
-// 2^x on the FMA / integer pipes (keeps the SFU free).  Cody-Waite style range
-// reduction x = n + f, n = round(x) taken from the low mantissa bits of
-// x + 1.5 * 2^23, f in [-1/2, 1/2]; 2^f by the cubic 1 + f (c1 + f (c2 + f c3))
-// fitted here to 2^f on [-1/2, 1/2] for least maximum relative error
-// (Lawson-weighted least squares; max relative error 1.02e-4, below the bf16
-// rounding of P).  n is added to the exponent field.  x is clamped at -127,
-// where the result is exactly +0 (p(0) = 1), so masked scores give 0.
-__device__ __forceinline__ float ex2_fma(float x) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c1 = 0.6932829022f, c2 = 0.2422103733f, c3 = 0.0550085828f;
-  x = fmaxf(x, -127.0f);
-  const float t = x + kShift;
-  const float f = x - (t - kShift);
-  const float p = fmaf(f, fmaf(f, fmaf(f, c3, c2), c1), 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// 2^x on the FMA / integer pipes for two values at once (keeps the SFU free).
+// Cody-Waite style range reduction x = n + f, n = round(x) taken from the low
+// mantissa bits of x + 1.5 * 2^23, f in [-1/2, 1/2]; 2^f by the cubic
+// 1 + f (c1 + f (c2 + f c3)) fitted here to 2^f on [-1/2, 1/2] for least
+// maximum relative error (Lawson-weighted least squares; max relative error
+// 1.02e-4, below the bf16 rounding of P); n is added to the exponent field.
+// x is clamped at -127, where the result is exactly +0 (p(0) = 1), so masked
+// scores give 0.  The arithmetic uses packed fp32x2 instructions.
+constexpr float kExpC1 = 0.6932829022f, kExpC2 = 0.2422103733f, kExpC3 = 0.0550085828f;
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+  const float2 kShift = make_float2(12582912.0f, 12582912.0f);
+  const float2 kNegShift = make_float2(-12582912.0f, -12582912.0f);
+  const float2 one = make_float2(1.0f, 1.0f);
+  const float2 c1 = make_float2(kExpC1, kExpC1);
+  const float2 c2 = make_float2(kExpC2, kExpC2);
+  const float2 c3 = make_float2(kExpC3, kExpC3);
+  x.x = fmaxf(x.x, -127.0f);
+  x.y = fmaxf(x.y, -127.0f);
+  const float2 t = fadd2(x, kShift);
+  const float2 n = fadd2(t, kNegShift);
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+  const float2 p = ffma2(f, ffma2(f, ffma2(f, c3, c2), c1), one);
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -374,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           umma_ts(d, pa + kk * 8, sdesc_sw128(vb + kk * 16 * 128, L::kBoxBytes, 1024), kIdescO,
                   (j > 0 || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_bar(&ctl->q_full, 0, ctl) && wait_bar(&ctl->k_full[0], 0, ctl);
+      bool ok = spin_bar(&ctl->q_full, 0, ctl) && spin_bar(&ctl->k_full[0], 0, ctl);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -387,12 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const int st = j % kStages;
         const bool more = j + 1 < n_tiles;
         // tile 0: PV_0(j), then S_0(j+1)
-        if (!(ok = wait_bar(&ctl->p_full[0], (uint32_t)j & 1u, ctl))) break;
-        if (!(ok = wait_bar(&ctl->v_full[st], (uint32_t)(j / kStages) & 1u, ctl))) break;
+        if (!(ok = spin_bar(&ctl->p_full[0], (uint32_t)j & 1u, ctl))) break;
+        if (!(ok = spin_bar(&ctl->v_full[st], (uint32_t)(j / kStages) & 1u, ctl))) break;
         tc_fence_after();
         issue_pv(0, j);
         if (more) {
-          if (!(ok = wait_bar(&ctl->k_full[(j + 1) % kStages],
+          if (!(ok = spin_bar(&ctl->k_full[(j + 1) % kStages],
                               (uint32_t)((j + 1) / kStages) & 1u, ctl)))
             break;
           tc_fence_after();
@@ -402,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           umma_commit(&ctl->o_done[0]);
         }
         // tile 1: PV_1(j), then S_1(j+1)
-        if (!(ok = wait_bar(&ctl->p_full[1], (uint32_t)j & 1u, ctl))) break;
+        if (!(ok = spin_bar(&ctl->p_full[1], (uint32_t)j & 1u, ctl))) break;
         tc_fence_after();
         issue_pv(1, j);
         umma_commit(&ctl->v_empty[st]);
@@ -472,13 +503,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             if (!((keep >> n) & 1u)) s[32 * c + n] = __float_as_uint(-INFINITY);
         }
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+      float mx[16];                                 // 16 independent chains, then a tree
 #pragma unroll
-      for (int n = 0; n < 128; n += 2) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[n]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[n + 1]));
-      }
-      const float m_new = fmaxf(m_ref, fmaxf(mx0, mx1) * sl2);
+      for (int k = 0; k < 16; ++k) mx[k] = __uint_as_float(s[k]);
+#pragma unroll
+      for (int n = 16; n < 128; n += 16)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(s[n + k]));
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int k = 0; k < w; ++k) mx[k] = fmaxf(mx[k], mx[k + w]);
+      const float m_new = fmaxf(m_ref, mx[0] * sl2);
 
       // O_t is stable here: S_t(j) was committed after PV_t(j-1).
       const bool grow = m_new > m_ref + kRescaleLog2;
@@ -499,30 +535,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (m_new != -INFINITY) m_ref = m_new;
       }
       const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float l0 = 0.f, l1 = 0.f;
+      const float2 sl2x2 = make_float2(sl2, sl2);
+      const float2 negm = make_float2(-msub, -msub);
+      float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {                 // 4 groups of 32 keys -> 16 packed columns
         uint32_t packed[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float x0 = fmaf(__uint_as_float(s[32 * c + 2 * e]), sl2, -msub);
-          const float x1 = fmaf(__uint_as_float(s[32 * c + 2 * e + 1]), sl2, -msub);
-          float p0, p1;
-          if (e >= 12) {                             // a quarter of the exps on the FMA pipe
-            p0 = ex2_fma(x0);
-            p1 = ex2_fma(x1);
+          const float2 sv = make_float2(__uint_as_float(s[32 * c + 2 * e]),
+                                        __uint_as_float(s[32 * c + 2 * e + 1]));
+          const float2 x = ffma2(sv, sl2x2, negm);
+          float2 pv;
+          if (e >= kExpSfuPairs) {                   // this share of the exps on the FMA pipe
+            pv = ex2_fma2(x);
           } else {
-            p0 = ex2_sfu(x0);
-            p1 = ex2_sfu(x1);
+            pv = make_float2(ex2_sfu(x.x), ex2_sfu(x.y));
           }
-          l0 += p0;
-          l1 += p1;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          lacc[e & 1] = fadd2(lacc[e & 1], pv);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(pv.x, pv.y);
           packed[e] = *reinterpret_cast<uint32_t*>(&b2);
         }
         tmem_st_32x32b_x16(s_addr + c * 16, packed);
       }
-      l_sum += l0 + l1;
+      l_sum += (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctl->p_full[tq]);

@@ -13,7 +13,7 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 
 def _coeffs():
     text = open(SRC).read()
-    m = re.search(r"c1 = ([0-9.e-]+)f, c2 = ([0-9.e-]+)f, c3 = ([0-9.e-]+)f", text)
+    m = re.search(r"kExpC1 = ([0-9.e-]+)f, kExpC2 = ([0-9.e-]+)f, kExpC3 = ([0-9.e-]+)f", text)
     return [np.float32(float(x)) for x in m.groups()]
 
 
