@@ -62,7 +62,7 @@ constexpr int kWarpMma = 9;
 constexpr float kRescaleLog2 = 8.0f;
 // Of the 16 key pairs in each 32-key group, pairs [0, kExpSfuPairs) take exp2 on
 // the SFU and the rest on the FMA pipe.
-constexpr int kExpSfuPairs = 12;
+constexpr int kExpSfuPairs = 16;
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S_t / P_t at t * 128, O_t at 256 + t * 128.
 constexpr uint32_t kTmemS = 0;
