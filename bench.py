@@ -157,6 +157,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ---------------------------------------------------------- multi-process --
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of every rank's value (the whole job ends when the slowest rank does)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(world: int, steps: int, flops_per_step: float, elapsed_ms: float) -> float:
+    """TFLOP/s of all ranks together: every rank runs `steps` steps of its own work."""
+    return world * steps * flops_per_step / (elapsed_ms * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------- ours --
 
 def run_ours(args, rank: int, world: int, dist) -> dict:
@@ -218,11 +235,7 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
         dist.barrier()
     launches = kvcr.kvcr_launch_count() - launches0
     clocks = sampler.stop()
-    elapsed_ms = ev0.elapsed_time(ev1)
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
 
     # ---------------- per-kernel times (traced pass, same steps) ----------------
     kvcr.kvcr_trace_reset()
@@ -268,16 +281,12 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     kvcr.kvcr_check_status()
 
     flops = step_flops(spec)
-    value = world * args.steps * flops / (elapsed_ms * 1e-3) / 1e12
-    e2e_value = world * args.steps * flops / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_throughput(world, args.steps, flops, elapsed_ms)
+    e2e_value = whole_job_throughput(world, args.steps, flops, e2e_ms)
     peaks, peak_kind = load_peaks()
     attn = kt.get("chunk_attn", {})
     attn_ms = attn.get("avg_ms", float("nan"))
@@ -364,13 +373,17 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def cpu_baseline(budget_s: float = 12.0) -> dict:
-    run, flops, n = oracle_sample(32)
-    t0 = time.perf_counter()
-    run()
-    t1 = time.perf_counter() - t0
-    per_row = t1 / n
-    rows = int(max(32, min(2048, budget_s / max(per_row, 1e-6))))
+def cpu_baseline(budget_s: float = 15.0) -> dict:
+    # two probe sizes separate the fixed cost (RoPE of the chunk's keys) from the per-row cost
+    times = []
+    for n_probe in (32, 128):
+        run, flops, n = oracle_sample(n_probe)
+        t0 = time.perf_counter()
+        run()
+        times.append((n, time.perf_counter() - t0))
+    per_row = max((times[1][1] - times[0][1]) / (times[1][0] - times[0][0]), 1e-6)
+    fixed = max(times[0][1] - per_row * times[0][0], 0.0)
+    rows = int(max(32, min(SPEC.chunk_tokens, (budget_s - fixed) / per_row)))
     run, flops, n = oracle_sample(rows)
     t0 = time.perf_counter()
     run()

@@ -214,6 +214,15 @@ int kvcr_check_status(void *stream);
 
 const char *kvcr_last_error(void);
 
+/* Failure-path test hook (for tests; off by default).  kind = 1 makes every
+ * later tensor-core attention launch withhold one internal "P ready" signal, so
+ * a wait inside the kernel runs out: the kernel then records KVCR_ETIMEOUT (read
+ * with kvcr_check_status), drains its in-flight copies and MMAs, frees its
+ * tensor memory and returns with its outputs invalid; the CUDA context stays
+ * usable.  kind = 0 turns it off.  wait_ns > 0 replaces the 2 s bound of every
+ * device wait of those launches (0 restores it). */
+int kvcr_debug_inject(int kind, long long wait_ns);
+
 /* -------------------------------------------------------------- trace ---- */
 
 /* Kernel ids for tracing. */

@@ -77,6 +77,7 @@ struct __align__(8) Ctl {
   int abort;
   int n_tiles;
   int pad;
+  unsigned long long wait_ns;  // bound of every wait (from the launch parameters)
   uint16_t tiles[kMobaMaxTiles];  // MoBA: key tile | class(tile 0) << 12 | class(tile 1) << 14
 };
 
@@ -139,7 +140,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Ctl* ct
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
     if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
-    if (globaltimer() - t0 > (uint64_t)kWaitTimeoutNs) {
+    if (globaltimer() - t0 > ctl->wait_ns) {
       atomicExch(&g_attn_status, (int)KVCR_ETIMEOUT);
       *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
       return false;
@@ -157,7 +158,7 @@ __device__ __forceinline__ bool spin_bar(uint64_t* bar, uint32_t parity, Ctl* ct
   while (!mbar_test_wait(bar, parity)) {
     if ((++n & 255u) == 0u) {
       if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
-      if (globaltimer() - t0 > (uint64_t)kWaitTimeoutNs) {
+      if (globaltimer() - t0 > ctl->wait_ns) {
         atomicExch(&g_attn_status, (int)KVCR_ETIMEOUT);
         *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
         return false;
@@ -317,6 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
+    ctl->wait_ns = p.c.wait_ns > 0 ? (unsigned long long)p.c.wait_ns
+                                   : (unsigned long long)kWaitTimeoutNs;
     if constexpr (!kMoba) ctl->n_tiles = p.s.n_vis * p.s.tiles_per_slot + p.s.cur_tiles;
     fence_mbar_init();
   }
@@ -561,7 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       l_sum += (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&ctl->p_full[tq]);
+      // test hook: tile 1 withholds its first P-ready arrival, so the MMA issuer's
+      // wait runs out and the whole CTA takes the timeout path
+      if (!(p.c.inject == 1 && tq == 1 && j == 0)) mbar_arrive(&ctl->p_full[tq]);
     }
 
     // ---------------------------------------------------------- epilogue --

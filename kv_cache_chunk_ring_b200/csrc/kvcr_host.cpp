@@ -68,13 +68,14 @@ EncodeTiledFn encode_fn() {
 }
 
 // Tiled map over a bf16 tensor [..][tokens][H][D] (innermost first: D, H,
-// tokens[, slots]); box = 64 x 1 x 128 (x 1), 128-byte swizzle, zero fill.
-int encode_bf16_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims) {
+// tokens[, slots]); box = 64 x 1 x box_rows (x 1), 128-byte swizzle, zero fill.
+int encode_bf16_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                    int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(KVCR_ECUDA, "cuTensorMapEncodeTiled not available from the driver");
   cuuint64_t gdim[4];
   cuuint64_t gstride[3];
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)kTile, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   uint64_t stride = 2;
   for (int i = 0; i < rank; ++i) {
@@ -90,6 +91,10 @@ int encode_bf16_map(CUtensorMap* m, const void* base, int rank, const uint64_t* 
                                                      std::to_string((int)r) + ")");
   return KVCR_OK;
 }
+
+// --------------------------------------------------------- failure hook --
+std::atomic<int> g_inject_kind{0};
+std::atomic<long long> g_inject_wait_ns{0};
 
 // ----------------------------------------------------------------- tracing --
 std::atomic<long long> g_launches{0};
@@ -207,6 +212,10 @@ struct kvcr_cache {
   int last_frame;
   std::vector<int> last_slots, last_evicted;
 };
+
+namespace kvcr {
+InjectState inject_state() { return InjectState{g_inject_kind.load(), g_inject_wait_ns.load()}; }
+}  // namespace kvcr
 
 namespace {
 
@@ -398,8 +407,8 @@ int kv_cache_init(kvcr_cache** out, int sinks, int window, int tokens_per_frame,
     if (dtype == KVCR_BF16) {
       const uint64_t dims[4] = {(uint64_t)head_dim, (uint64_t)heads, (uint64_t)tokens_per_frame,
                                 (uint64_t)(sinks + window)};
-      int rc = encode_bf16_map(&c->tm_kc, c->storage + L.k_off, 4, dims);
-      if (!rc) rc = encode_bf16_map(&c->tm_vc, c->storage + L.v_off, 4, dims);
+      int rc = encode_bf16_map(&c->tm_kc, c->storage + L.k_off, 4, dims, kKeyTile);
+      if (!rc) rc = encode_bf16_map(&c->tm_vc, c->storage + L.v_off, 4, dims, kKeyTile);
       if (rc) {
         delete c;
         return rc;
@@ -593,9 +602,9 @@ int chunk_attention_fwd(kvcr_cache* c, const void* q, int n_q, const void* k_cur
     std::memset(&p, 0, sizeof(p));
     const uint64_t dq[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_q};
     const uint64_t dn[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_cur};
-    rc = encode_bf16_map(&p.tm_q, q_src, 3, dq);
-    if (!rc) rc = encode_bf16_map(&p.tm_kn, k_src, 3, dn);
-    if (!rc) rc = encode_bf16_map(&p.tm_vn, v_cur, 3, dn);
+    rc = encode_bf16_map(&p.tm_q, q_src, 3, dq, kTile);
+    if (!rc) rc = encode_bf16_map(&p.tm_kn, k_src, 3, dn, kKeyTile);
+    if (!rc) rc = encode_bf16_map(&p.tm_vn, v_cur, 3, dn, kKeyTile);
     if (rc) return rc;
     p.tm_kc = c->tm_kc;
     p.tm_vc = c->tm_vc;
@@ -604,11 +613,13 @@ int chunk_attention_fwd(kvcr_cache* c, const void* q, int n_q, const void* k_cur
     p.c.n_q = n_q;
     p.c.H = c->H;
     p.c.scale_log2 = (float)(scale * 1.4426950408889634);
+    p.c.inject = inject_state().kind;
+    p.c.wait_ns = inject_state().wait_ns;
     p.s.T = c->T;
     p.s.n_vis = n_vis;
-    p.s.tiles_per_slot = (c->T + kTile - 1) / kTile;
+    p.s.tiles_per_slot = (c->T + kKeyTile - 1) / kKeyTile;
     p.s.n_cur = n_cur;
-    p.s.cur_tiles = (n_cur + kTile - 1) / kTile;
+    p.s.cur_tiles = (n_cur + kKeyTile - 1) / kKeyTile;
     for (int i = 0; i < n_vis; ++i) p.s.slots[i] = slots[i];
     cudaError_t e;
     {
@@ -725,9 +736,9 @@ int chunk_attention_fwd_static_scratch(kvcr_cache* c, const void* q, int n_q, co
     std::memset(&p, 0, sizeof(p));
     const uint64_t dq[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_q};
     const uint64_t dn[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_cur};
-    rc = encode_bf16_map(&p.tm_q, q_src, 3, dq);
-    if (!rc) rc = encode_bf16_map(&p.tm_kn, k_src, 3, dn);
-    if (!rc) rc = encode_bf16_map(&p.tm_vn, v_cur, 3, dn);
+    rc = encode_bf16_map(&p.tm_q, q_src, 3, dq, kTile);
+    if (!rc) rc = encode_bf16_map(&p.tm_kn, k_src, 3, dn, kKeyTile);
+    if (!rc) rc = encode_bf16_map(&p.tm_vn, v_cur, 3, dn, kKeyTile);
     if (rc) return rc;
     p.tm_kc = c->tm_kc;
     p.tm_vc = c->tm_vc;
@@ -736,11 +747,13 @@ int chunk_attention_fwd_static_scratch(kvcr_cache* c, const void* q, int n_q, co
     p.c.n_q = n_q;
     p.c.H = c->H;
     p.c.scale_log2 = (float)(scale * 1.4426950408889634);
+    p.c.inject = inject_state().kind;
+    p.c.wait_ns = inject_state().wait_ns;
     p.s.T = c->T;
     p.s.n_vis = n_vis;
-    p.s.tiles_per_slot = (c->T + kTile - 1) / kTile;
+    p.s.tiles_per_slot = (c->T + kKeyTile - 1) / kKeyTile;
     p.s.n_cur = n_cur;
-    p.s.cur_tiles = (n_cur + kTile - 1) / kTile;
+    p.s.cur_tiles = (n_cur + kKeyTile - 1) / kKeyTile;
     for (int i = 0; i < n_vis; ++i) p.s.slots[i] = slots[i];
     cudaError_t e;
     {
@@ -878,9 +891,9 @@ int moba_attention_fwd(const void* q, const void* k, const void* v,
     for (size_t i = 0; i < last_order.size(); ++i) p->s.order[i] = last_order[i];
   }
   const uint64_t d3[3] = {(uint64_t)head_dim, (uint64_t)heads, (uint64_t)l.L};
-  rc = encode_bf16_map(&p->tm_q, q, 3, d3);
-  if (!rc) rc = encode_bf16_map(&p->tm_k, k, 3, d3);
-  if (!rc) rc = encode_bf16_map(&p->tm_v, v, 3, d3);
+  rc = encode_bf16_map(&p->tm_q, q, 3, d3, kTile);
+  if (!rc) rc = encode_bf16_map(&p->tm_k, k, 3, d3, kKeyTile);
+  if (!rc) rc = encode_bf16_map(&p->tm_v, v, 3, d3, kKeyTile);
   if (rc) {
     delete p;
     return rc;
@@ -891,6 +904,8 @@ int moba_attention_fwd(const void* q, const void* k, const void* v,
   p->c.n_q = l.L;
   p->c.H = heads;
   p->c.scale_log2 = (float)(scale * 1.4426950408889634);
+  p->c.inject = inject_state().kind;
+  p->c.wait_ns = inject_state().wait_ns;
   p->s.n_chunks = l.n;
   p->s.chunk_tokens = l.c;
   p->s.n_bidir = l.m;
@@ -919,6 +934,13 @@ int kvcr_check_status(void* stream) {
 }
 
 long long kvcr_launch_count(void) { return g_launches.load(); }
+
+int kvcr_debug_inject(int kind, long long wait_ns) {
+  if (kind < 0 || kind > 1 || wait_ns < 0) return fail(KVCR_EINVAL, "kvcr_debug_inject: bad argument");
+  g_inject_kind.store(kind);
+  g_inject_wait_ns.store(wait_ns);
+  return KVCR_OK;
+}
 
 int kvcr_trace_enable(int on) {
   std::lock_guard<std::mutex> g(g_trace_mu);

@@ -13,7 +13,8 @@ namespace kvcr {
 constexpr int kMaxSlots = 32;        // sinks + window
 constexpr int kMaxFrames = 16;       // frames of one append / one current chunk
 constexpr int kMaxPairsT = 32;       // rotary pairs on the t axis
-constexpr int kTile = 128;           // rows / keys per attention tile
+constexpr int kTile = 128;           // query rows per attention tile (MoBA class granularity)
+constexpr int kKeyTile = 128;        // keys per K / V tile of the attention kernel
 constexpr int kMobaMaxTiles = 4096;  // MoBA sequence length <= 4096 * 128 tokens
 constexpr long long kWaitTimeoutNs = 2000000000LL;  // bounded device waits: 2 s
 
@@ -61,8 +62,17 @@ struct AttnCommon {
   float* lse;
   int n_q;
   int H;
-  float scale_log2;  // softmax scale * log2(e)
+  float scale_log2;   // softmax scale * log2(e)
+  int inject;         // test hook: 1 = one P-ready arrival is never made (a wait runs out)
+  long long wait_ns;  // bound of every device wait
 };
+
+// Test hook for the failure path (set by kvcr_debug_inject, read at launch).
+struct InjectState {
+  int kind;
+  long long wait_ns;
+};
+InjectState inject_state();
 
 struct ChunkAttnParams {
   CUtensorMap tm_q;   // 3D (D, H, n_q)

@@ -33,8 +33,8 @@ EXPORTS = [
     "kv_cache_slot_map", "kv_cache_last_append", "kv_cache_num_cached", "kv_cache_slot_data",
     "kv_cache_destroy",
     "chunk_attention_fwd", "chunk_attention_fwd_static_scratch", "moba_attention_fwd", "moba_classify_tiles", "kvcr_check_status",
-    "kvcr_last_error", "kvcr_launch_count", "kvcr_trace_enable", "kvcr_trace_reset",
-    "kvcr_trace_read",
+    "kvcr_last_error", "kvcr_launch_count", "kvcr_debug_inject", "kvcr_trace_enable",
+    "kvcr_trace_reset", "kvcr_trace_read",
 ]
 
 
@@ -89,6 +89,7 @@ def lib() -> ctypes.CDLL:
         "kvcr_check_status": (c_int, [c_p]),
         "kvcr_last_error": (ctypes.c_char_p, []),
         "kvcr_launch_count": (ctypes.c_longlong, []),
+        "kvcr_debug_inject": (c_int, [c_int, ctypes.c_longlong]),
         "kvcr_trace_enable": (c_int, [c_int]),
         "kvcr_trace_reset": (c_int, []),
         "kvcr_trace_read": (c_int, [c_int, ctypes.POINTER(ctypes.c_longlong),
@@ -241,6 +242,11 @@ def kvcr_check_status(stream=None) -> None:
 
 def kvcr_launch_count() -> int:
     return int(lib().kvcr_launch_count())
+
+
+def kvcr_debug_inject(kind: int, wait_ns: int = 0) -> None:
+    """Failure-path test hook (see include/kvcr.h); kind 0 turns it off."""
+    _check(lib().kvcr_debug_inject(int(kind), int(wait_ns)))
 
 
 def kvcr_trace_enable(on: bool) -> None:
