@@ -479,6 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
 
     for (int j = 0; j < n_tiles; ++j) {
+      const TileRef t = tile_ref(p, ctl, j);        // independent of S: before the wait
       ok = wait_bar(&ctl->s_full[tq], (uint32_t)j & 1u, ctl);
       if (!__all_sync(0xFFFFFFFFu, ok)) {  // leave the loop warp-uniformly
         ok = false;
@@ -492,7 +493,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       tmem_ld_32x32b_x32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_ld_wait();
 
-      const TileRef t = tile_ref(p, ctl, j);
       const int cls = tq == 0 ? t.cls0 : t.cls1;
       if (t.valid < kTile || (kMoba && cls != kTileFull)) {
 #pragma unroll
@@ -540,7 +540,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
       const float2 sl2x2 = make_float2(sl2, sl2);
       const float2 negm = make_float2(-msub, -msub);
-      float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {                 // 4 groups of 32 keys -> 16 packed columns
         uint32_t packed[16];
@@ -555,18 +554,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           } else {
             pv = make_float2(ex2_sfu(x.x), ex2_sfu(x.y));
           }
-          lacc[e & 1] = fadd2(lacc[e & 1], pv);
+          s[32 * c + 2 * e] = __float_as_uint(pv.x); // kept for the row sum below
+          s[32 * c + 2 * e + 1] = __float_as_uint(pv.y);
           __nv_bfloat162 b2 = __floats2bfloat162_rn(pv.x, pv.y);
           packed[e] = *reinterpret_cast<uint32_t*>(&b2);
         }
         tmem_st_32x32b_x16(s_addr + c * 16, packed);
       }
-      l_sum += (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
       tmem_st_wait();
       tc_fence_before();
       // test hook: tile 1 withholds its first P-ready arrival, so the MMA issuer's
       // wait runs out and the whole CTA takes the timeout path
       if (!(p.c.inject == 1 && tq == 1 && j == 0)) mbar_arrive(&ctl->p_full[tq]);
+      // the row sum is off the path to the MMA: accumulated after P is released
+      float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int n = 0; n < 128; n += 2)
+        lacc[(n >> 1) & 3] = fadd2(lacc[(n >> 1) & 3],
+                                   make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])));
+      l_sum += ((lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y)) +
+               ((lacc[2].x + lacc[2].y) + (lacc[3].x + lacc[3].y));
     }
 
     // ---------------------------------------------------------- epilogue --
