@@ -27,8 +27,9 @@
 //               is written only after PV_t(j) has read P_t(j).
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r owns
 //               query row r = TMEM lane r, so the row max / sum stay in-thread;
-//               exp2 with the scale folded in, part of it evaluated on the FMA
-//               pipe (range reduction + cubic, packed fp32x2) to offload the SFU; the
+//               exp2 with the scale folded in (packed fp32x2 arithmetic); P is
+//               released to the MMA in two 64-key halves and the row sum is
+//               accumulated after the release, off the path to the MMA; the
 //               running max only moves (and O_t is rescaled in TMEM) when it
 //               grows by more than 2^8, and the final normalisation uses the same
 //               stale max, so the result is exact.
@@ -71,7 +72,7 @@ constexpr uint32_t kTmemO = 256;
 struct __align__(8) Ctl {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t s_full[2], p_full[2][2], o_done[2];  // p_full[tile][key half]
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -313,7 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&ctl->s_full[t], 1);
-      mbar_init(&ctl->p_full[t], 128);
+      mbar_init(&ctl->p_full[t][0], 128);
+      mbar_init(&ctl->p_full[t][1], 128);
       mbar_init(&ctl->o_done[t], 1);
     }
     mbar_init(&ctl->drain, 1);
@@ -398,15 +400,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                   kk > 0 ? 1u : 0u);
         }
       };
-      // O_t += P_t(j) V_j, P_t in TMEM (8 packed columns per 16 keys)
-      auto issue_pv = [&](int t, int j) {
+      // O_t += P_t(j) V_j over keys [64 hf, 64 hf + 64), P_t in TMEM (8 packed
+      // columns per 16 keys)
+      auto issue_pv = [&](int t, int j, int hf) {
         const uint32_t pa = tmem + kTmemS + (uint32_t)t * 128u;
         const uint32_t d = tmem + kTmemO + (uint32_t)t * 128u;
         const uint32_t vb = sV + (j % kStages) * L::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * hf + k4;
           umma_ts(d, pa + kk * 8, sdesc_sw128(vb + kk * 16 * 128, L::kBoxBytes, 1024), kIdescO,
                   (j > 0 || kk > 0) ? 1u : 0u);
+        }
       };
       bool ok = spin_bar(&ctl->q_full, 0, ctl) && spin_bar(&ctl->k_full[0], 0, ctl);
       if (ok) {
@@ -420,11 +425,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j % kStages;
         const bool more = j + 1 < n_tiles;
-        // tile 0: PV_0(j), then S_0(j+1)
-        if (!(ok = spin_bar(&ctl->p_full[0], (uint32_t)j & 1u, ctl))) break;
+        // tile 0: PV_0(j) half by half as P arrives, then S_0(j+1)
         if (!(ok = spin_bar(&ctl->v_full[st], (uint32_t)(j / kStages) & 1u, ctl))) break;
+        if (!(ok = spin_bar(&ctl->p_full[0][0], (uint32_t)j & 1u, ctl))) break;
         tc_fence_after();
-        issue_pv(0, j);
+        issue_pv(0, j, 0);
+        if (!(ok = spin_bar(&ctl->p_full[0][1], (uint32_t)j & 1u, ctl))) break;
+        tc_fence_after();
+        issue_pv(0, j, 1);
         if (more) {
           if (!(ok = spin_bar(&ctl->k_full[(j + 1) % kStages],
                               (uint32_t)((j + 1) / kStages) & 1u, ctl)))
@@ -436,9 +444,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           umma_commit(&ctl->o_done[0]);
         }
         // tile 1: PV_1(j), then S_1(j+1)
-        if (!(ok = spin_bar(&ctl->p_full[1], (uint32_t)j & 1u, ctl))) break;
+        if (!(ok = spin_bar(&ctl->p_full[1][0], (uint32_t)j & 1u, ctl))) break;
         tc_fence_after();
-        issue_pv(1, j);
+        issue_pv(1, j, 0);
+        if (!(ok = spin_bar(&ctl->p_full[1][1], (uint32_t)j & 1u, ctl))) break;
+        tc_fence_after();
+        issue_pv(1, j, 1);
         umma_commit(&ctl->v_empty[st]);
         if (more) {
           issue_s(1, j + 1);
@@ -560,12 +571,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           packed[e] = *reinterpret_cast<uint32_t*>(&b2);
         }
         tmem_st_32x32b_x16(s_addr + c * 16, packed);
+        if (c & 1) {                                // keys [64 (c/2), 64 (c/2) + 64) are ready
+          tmem_st_wait();
+          tc_fence_before();
+          // test hook: tile 1 withholds its first P-ready arrival, so the MMA issuer's
+          // wait runs out and the whole CTA takes the timeout path
+          if (!(p.c.inject == 1 && tq == 1 && j == 0 && c == 1))
+            mbar_arrive(&ctl->p_full[tq][c >> 1]);
+        }
       }
-      tmem_st_wait();
-      tc_fence_before();
-      // test hook: tile 1 withholds its first P-ready arrival, so the MMA issuer's
-      // wait runs out and the whole CTA takes the timeout path
-      if (!(p.c.inject == 1 && tq == 1 && j == 0)) mbar_arrive(&ctl->p_full[tq]);
       // the row sum is off the path to the MMA: accumulated after P is released
       float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};
