@@ -61,6 +61,8 @@ constexpr uint32_t kRegsSoftmax = 208;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr float kRescaleLog2 = 8.0f;
+// P of a tile is released to the MMA in this many parts of 128 / kPParts keys.
+constexpr int kPParts = 2;
 // Of the 16 key pairs in each 32-key group, pairs [0, kExpSfuPairs) take exp2 on
 // the SFU and the rest on the FMA pipe.
 constexpr int kExpSfuPairs = 16;
@@ -72,7 +74,7 @@ constexpr uint32_t kTmemO = 256;
 struct __align__(8) Ctl {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2][2], o_done[2];  // p_full[tile][key half]
+  uint64_t s_full[2], p_full[2][kPParts], o_done[2];  // p_full[tile][key part]
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -314,8 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&ctl->s_full[t], 1);
-      mbar_init(&ctl->p_full[t][0], 128);
-      mbar_init(&ctl->p_full[t][1], 128);
+      for (int q = 0; q < kPParts; ++q) mbar_init(&ctl->p_full[t][q], 128);
       mbar_init(&ctl->o_done[t], 1);
     }
     mbar_init(&ctl->drain, 1);
@@ -400,15 +401,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                   kk > 0 ? 1u : 0u);
         }
       };
-      // O_t += P_t(j) V_j over keys [64 hf, 64 hf + 64), P_t in TMEM (8 packed
-      // columns per 16 keys)
+      // O_t += P_t(j) V_j over part hf of the keys, P_t in TMEM (8 packed columns
+      // per 16 keys)
       auto issue_pv = [&](int t, int j, int hf) {
         const uint32_t pa = tmem + kTmemS + (uint32_t)t * 128u;
         const uint32_t d = tmem + kTmemO + (uint32_t)t * 128u;
         const uint32_t vb = sV + (j % kStages) * L::kTileBytes;
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const int kk = 4 * hf + k4;
+        for (int k4 = 0; k4 < 8 / kPParts; ++k4) {
+          const int kk = (8 / kPParts) * hf + k4;
           umma_ts(d, pa + kk * 8, sdesc_sw128(vb + kk * 16 * 128, L::kBoxBytes, 1024), kIdescO,
                   (j > 0 || kk > 0) ? 1u : 0u);
         }
@@ -427,12 +428,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const bool more = j + 1 < n_tiles;
         // tile 0: PV_0(j) half by half as P arrives, then S_0(j+1)
         if (!(ok = spin_bar(&ctl->v_full[st], (uint32_t)(j / kStages) & 1u, ctl))) break;
-        if (!(ok = spin_bar(&ctl->p_full[0][0], (uint32_t)j & 1u, ctl))) break;
-        tc_fence_after();
-        issue_pv(0, j, 0);
-        if (!(ok = spin_bar(&ctl->p_full[0][1], (uint32_t)j & 1u, ctl))) break;
-        tc_fence_after();
-        issue_pv(0, j, 1);
+        for (int q = 0; ok && q < kPParts; ++q) {
+          if (!(ok = spin_bar(&ctl->p_full[0][q], (uint32_t)j & 1u, ctl))) break;
+          tc_fence_after();
+          issue_pv(0, j, q);
+        }
+        if (!ok) break;
         if (more) {
           if (!(ok = spin_bar(&ctl->k_full[(j + 1) % kStages],
                               (uint32_t)((j + 1) / kStages) & 1u, ctl)))
@@ -444,12 +445,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           umma_commit(&ctl->o_done[0]);
         }
         // tile 1: PV_1(j), then S_1(j+1)
-        if (!(ok = spin_bar(&ctl->p_full[1][0], (uint32_t)j & 1u, ctl))) break;
-        tc_fence_after();
-        issue_pv(1, j, 0);
-        if (!(ok = spin_bar(&ctl->p_full[1][1], (uint32_t)j & 1u, ctl))) break;
-        tc_fence_after();
-        issue_pv(1, j, 1);
+        for (int q = 0; ok && q < kPParts; ++q) {
+          if (!(ok = spin_bar(&ctl->p_full[1][q], (uint32_t)j & 1u, ctl))) break;
+          tc_fence_after();
+          issue_pv(1, j, q);
+        }
+        if (!ok) break;
         umma_commit(&ctl->v_empty[st]);
         if (more) {
           issue_s(1, j + 1);
@@ -571,13 +572,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           packed[e] = *reinterpret_cast<uint32_t*>(&b2);
         }
         tmem_st_32x32b_x16(s_addr + c * 16, packed);
-        if (c & 1) {                                // keys [64 (c/2), 64 (c/2) + 64) are ready
+        if (((c + 1) % (4 / kPParts)) == 0) {       // part c / (4 / kPParts) of P is ready
           tmem_st_wait();
           tc_fence_before();
           // test hook: tile 1 withholds its first P-ready arrival, so the MMA issuer's
           // wait runs out and the whole CTA takes the timeout path
-          if (!(p.c.inject == 1 && tq == 1 && j == 0 && c == 1))
-            mbar_arrive(&ctl->p_full[tq][c >> 1]);
+          if (!(p.c.inject == 1 && tq == 1 && j == 0 && c == 4 / kPParts - 1))
+            mbar_arrive(&ctl->p_full[tq][c / (4 / kPParts)]);
         }
       }
       // the row sum is off the path to the MMA: accumulated after P is released
