@@ -200,6 +200,36 @@ int moba_attention_fwd(const void *q, const void *k, const void *v,
                        kvcr_dtype dtype, float softmax_scale, void *o, float *lse,
                        void *stream);
 
+/* Backward of moba_attention_fwd(): with P the forward's probabilities
+ * (recomputed from its LSE), dV = P^T dO, dP = dO V^T, D = rowsum(dO o O),
+ * dS = P o (dP - D), dQ = scale * dS K, dK = scale * dS^T Q, for the model
+ * trained under the MoBA mask ("Infinite Worlds with Versatile Interactions",
+ * causal-pretraining paragraph; "Mix Forcing", "Mix the training modes"; the
+ * pages print no backward pass, this is the chain rule through the forward).
+ *   q, k, v, o, d_o: device [L][heads][head_dim] bf16, 16-byte aligned; o and
+ *          lse are the forward's outputs for the same q, k, v, layout, scale.
+ *   lse:   device fp32 [heads][L] (natural log, as moba_attention_fwd writes).
+ *   dq, dk, dv: device [L][heads][head_dim] bf16, written in full (no
+ *          accumulation into previous contents).
+ *   workspace: caller-owned device buffer of at least
+ *          moba_attention_bwd_workspace_bytes() bytes, 16-byte aligned, used
+ *          as scratch for the duration of the call's GPU work (no initial
+ *          contents needed); calls whose GPU work overlaps need separate ones.
+ * Three kernels run on `stream`, no atomics: the result does not depend on
+ * scheduling.  Errors: KVCR_EINVAL (NULL / misaligned pointer), KVCR_ESHAPE,
+ * KVCR_ESTORAGE (workspace too small), KVCR_EUNSUPPORTED (dtype other than
+ * bf16, head_dim other than 64 / 128, GPU other than sm_100); nothing is
+ * launched on error. */
+int moba_attention_bwd(const void *q, const void *k, const void *v, const void *o,
+                       const void *d_o, const float *lse, const kvcr_moba_layout *layout,
+                       int heads, int head_dim, kvcr_dtype dtype, float softmax_scale,
+                       void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/* Bytes of workspace moba_attention_bwd() needs: 8 per (head, row) with the
+ * rows rounded up to a multiple of 128; 0 for an invalid layout or heads < 1. */
+size_t moba_attention_bwd_workspace_bytes(const kvcr_moba_layout *layout, int heads);
+
 /* Host classification of the tile x tile blocks of the MoBA score matrix into
  * KVCR_TILE_EMPTY / PARTIAL / FULL (only in-range rows and columns count).
  * cls: host [nt * nt] row-major, nt = ceil(L / tile); cap = its length. */
@@ -215,8 +245,9 @@ int kvcr_check_status(void *stream);
 const char *kvcr_last_error(void);
 
 /* Failure-path test hook (for tests; off by default).  kind = 1 makes every
- * later tensor-core attention launch withhold one internal "P ready" signal, so
- * a wait inside the kernel runs out: the kernel then records KVCR_ETIMEOUT (read
+ * later tensor-core attention launch (forward and backward) withhold one
+ * internal "P ready" (or "dS ready") signal, so a wait inside the kernel runs
+ * out: the kernel then records KVCR_ETIMEOUT (read
  * with kvcr_check_status), drains its in-flight copies and MMAs, frees its
  * tensor memory and returns with its outputs invalid; the CUDA context stays
  * usable.  kind = 0 turns it off.  wait_ns > 0 replaces the 2 s bound of every
@@ -232,7 +263,10 @@ enum {
     KVCR_K_CHUNK_ATTN = 2,  /* tensor-core chunk attention (bf16) */
     KVCR_K_MOBA_ATTN = 3,   /* tensor-core MoBA attention (bf16) */
     KVCR_K_ATTN_F32 = 4,    /* fp32 CUDA-core attention */
-    KVCR_K_COUNT = 5
+    KVCR_K_MOBA_BWD_PREP = 5, /* MoBA backward: per-row LSE and rowsum(dO o O) */
+    KVCR_K_MOBA_BWD_DKDV = 6, /* MoBA backward: dK and dV (tensor cores) */
+    KVCR_K_MOBA_BWD_DQ = 7,   /* MoBA backward: dQ (tensor cores) */
+    KVCR_K_COUNT = 8
 };
 
 /* Count of every kernel the library launched in this process. */

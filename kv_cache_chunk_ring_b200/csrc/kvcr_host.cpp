@@ -28,6 +28,7 @@
 #include <string>
 #include <vector>
 
+#include "attn_bwd.h"
 #include "kvcr_internal.h"
 #include "moba_layout.h"
 #include "static_scratch.h"
@@ -818,40 +819,70 @@ int moba_classify_tiles(const kvcr_moba_layout* layout, int tile, uint8_t* cls, 
 }
 
 namespace {
-// Work units are pairs of 128-row query tiles (one CTA each).  A unit's work
-// is the number of key tiles hit by the union of its rows' allowed key
-// intervals; units are ordered heaviest first.
+// Number of 128-key tiles hit by the union of intervals [lo[k], hi[k]).
+int tiles_hit(const int* lo, const int* hi, int n) {
+  std::vector<std::pair<int, int>> iv;
+  for (int k = 0; k < n; ++k)
+    if (hi[k] > lo[k]) iv.push_back({lo[k] / kTile, (hi[k] - 1) / kTile});
+  std::sort(iv.begin(), iv.end());
+  int count = 0, cur_lo = -1, cur_hi = -2;
+  for (auto& t : iv) {
+    if (t.first > cur_hi) {
+      if (cur_hi >= cur_lo && cur_lo >= 0) count += cur_hi - cur_lo + 1;
+      cur_lo = t.first;
+      cur_hi = t.second;
+    } else {
+      cur_hi = std::max(cur_hi, t.second);
+    }
+  }
+  if (cur_lo >= 0) count += cur_hi - cur_lo + 1;
+  return count;
+}
+
+// Units ordered heaviest first (stable on ties).
+void order_by_work(const std::vector<int>& work, std::vector<uint16_t>& order) {
+  order.resize(work.size());
+  for (size_t i = 0; i < work.size(); ++i) order[i] = (uint16_t)i;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](uint16_t a, uint16_t b) { return work[a] > work[b]; });
+}
+
+// Forward work units are pairs of 128-row query tiles (one CTA each).  A unit's
+// work is the number of key tiles hit by the union of its rows' allowed key
+// intervals.
 void moba_order(const MobaLay& l, std::vector<uint16_t>& order) {
   constexpr int kUnitRows = 2 * kTile;
   const int nt = (l.L + kUnitRows - 1) / kUnitRows;
   std::vector<int> work(nt);
-  std::vector<std::pair<int, int>> iv;
   constexpr int kCap = 2 * kUnitRows + 8;
   int lo[kCap], hi[kCap];
   for (int i = 0; i < nt; ++i) {
     const int r0 = i * kUnitRows, r1 = std::min(r0 + kUnitRows, l.L);
-    const int n = moba_row_intervals(l, r0, r1, lo, hi, kCap);
-    iv.clear();
-    for (int k = 0; k < n; ++k)
-      if (hi[k] > lo[k]) iv.push_back({lo[k] / kTile, (hi[k] - 1) / kTile});
-    std::sort(iv.begin(), iv.end());
-    int count = 0, cur_lo = -1, cur_hi = -2;
-    for (auto& t : iv) {
-      if (t.first > cur_hi) {
-        if (cur_hi >= cur_lo && cur_lo >= 0) count += cur_hi - cur_lo + 1;
-        cur_lo = t.first;
-        cur_hi = t.second;
-      } else {
-        cur_hi = std::max(cur_hi, t.second);
-      }
-    }
-    if (cur_lo >= 0) count += cur_hi - cur_lo + 1;
-    work[i] = count;
+    work[i] = tiles_hit(lo, hi, moba_row_intervals(l, r0, r1, lo, hi, kCap));
   }
-  order.resize(nt);
-  for (int i = 0; i < nt; ++i) order[i] = (uint16_t)i;
-  std::stable_sort(order.begin(), order.end(),
-                   [&](uint16_t a, uint16_t b) { return work[a] > work[b]; });
+  order_by_work(work, order);
+}
+
+// Backward work units are single 128-row tiles: query tiles for dQ (work = key
+// tiles read), key tiles for dK / dV (work = query tiles that read them).
+void moba_bwd_orders(const MobaLay& l, std::vector<uint16_t>& by_query,
+                     std::vector<uint16_t>& by_key) {
+  const int nt = (l.L + kTile - 1) / kTile;
+  std::vector<int> wq(nt), wk(nt);
+  constexpr int kCap = 2 * kTile + 8;
+  int lo[kCap], hi[kCap];
+  for (int i = 0; i < nt; ++i) {
+    const int r0 = i * kTile, r1 = std::min(r0 + kTile, l.L);
+    wq[i] = tiles_hit(lo, hi, moba_row_intervals(l, r0, r1, lo, hi, kCap));
+    int n = 0, kk, ki, ks, ke;
+    for (int cp = r0; cp < r1 && n + 2 <= kCap; cp = ke) {
+      moba_block(l, cp, kk, ki, ks, ke);
+      n += moba_col_intervals(l, cp, lo + n, hi + n);
+    }
+    wk[i] = tiles_hit(lo, hi, n);
+  }
+  order_by_work(wq, by_query);
+  order_by_work(wk, by_key);
 }
 }  // namespace
 
@@ -922,14 +953,113 @@ int moba_attention_fwd(const void* q, const void* k, const void* v,
   return KVCR_OK;
 }
 
+size_t moba_attention_bwd_workspace_bytes(const kvcr_moba_layout* layout, int heads) {
+  MobaLay l;
+  if (moba_check_layout(layout, &l) != KVCR_OK || heads < 1) return 0;
+  const size_t lpad = (size_t)((l.L + kTile - 1) / kTile) * kTile;
+  return lpad * (size_t)heads * sizeof(float2);
+}
+
+int moba_attention_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const void* d_o, const float* lse, const kvcr_moba_layout* layout,
+                       int heads, int head_dim, kvcr_dtype dtype, float softmax_scale, void* dq,
+                       void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  MobaLay l;
+  int rc = moba_check_layout(layout, &l);
+  if (rc) return rc;
+  if (dtype != KVCR_BF16) return fail(KVCR_EUNSUPPORTED, "moba_attention_bwd: bf16 only");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(KVCR_EUNSUPPORTED, "moba_attention_bwd: head_dim must be 64 or 128");
+  if (heads < 1) return fail(KVCR_ESHAPE, "moba_attention_bwd: heads < 1");
+  if ((long long)l.L * heads * head_dim > (1LL << 31) - 1)
+    return fail(KVCR_ESHAPE, "moba_attention_bwd: tensor too large");
+  if (!q || !k || !v || !o || !d_o || !lse || !dq || !dk || !dv || !workspace)
+    return fail(KVCR_EINVAL, "moba_attention_bwd: NULL pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return fail(KVCR_EINVAL, "moba_attention_bwd: tensors and workspace must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(lse) & 3u)
+    return fail(KVCR_EINVAL, "moba_attention_bwd: lse must be 4-byte aligned");
+  if (workspace_bytes < moba_attention_bwd_workspace_bytes(layout, heads))
+    return fail(KVCR_ESTORAGE, "moba_attention_bwd: workspace smaller than "
+                               "moba_attention_bwd_workspace_bytes()");
+  int n_sm = 0, cc = 0;
+  rc = device_sm_count(&n_sm, &cc);
+  if (rc) return rc;
+  if (cc != 10) return fail(KVCR_EUNSUPPORTED, "moba_attention_bwd: needs an sm_100 GPU");
+
+  const int nt = (l.L + kTile - 1) / kTile;
+  static std::mutex mu;
+  static MobaLay last{0, 0, 0, 0};
+  static std::vector<uint16_t> by_query, by_key;
+  MobaBwdParams* p = new MobaBwdParams();
+  std::memset(p, 0, sizeof(*p));
+  const uint64_t d3[3] = {(uint64_t)head_dim, (uint64_t)heads, (uint64_t)l.L};
+  rc = encode_bf16_map(&p->tm_q, q, 3, d3, kTile);
+  if (!rc) rc = encode_bf16_map(&p->tm_k, k, 3, d3, kTile);
+  if (!rc) rc = encode_bf16_map(&p->tm_v, v, 3, d3, kTile);
+  if (!rc) rc = encode_bf16_map(&p->tm_do, d_o, 3, d3, kTile);
+  if (rc) {
+    delete p;
+    return rc;
+  }
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)head_dim);
+  float2* ws = static_cast<float2*>(workspace);
+  p->ws = ws;
+  p->dq = dq;
+  p->dk = dk;
+  p->dv = dv;
+  p->H = heads;
+  p->Lpad = nt * kTile;
+  p->scale = scale;
+  p->scale_log2 = (float)(scale * 1.4426950408889634);
+  p->inject = inject_state().kind;
+  p->wait_ns = inject_state().wait_ns;
+  p->s.n_chunks = l.n;
+  p->s.chunk_tokens = l.c;
+  p->s.n_bidir = l.m;
+  p->s.L = l.L;
+  p->s.n_units = nt;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MobaBwdPrepParams pp{o, d_o, lse, ws, l.L, nt * kTile, heads};
+  cudaError_t e;
+  {
+    LaunchScope scope(KVCR_K_MOBA_BWD_PREP, s);
+    e = launch_moba_bwd_prep(pp, head_dim, s);
+  }
+  if (e == cudaSuccess) {
+    std::lock_guard<std::mutex> g(mu);
+    if (!(last.n == l.n && last.c == l.c && last.m == l.m)) {
+      moba_bwd_orders(l, by_query, by_key);
+      last = l;
+    }
+    for (int i = 0; i < nt; ++i) p->s.order[i] = by_key[i];
+    {
+      LaunchScope scope(KVCR_K_MOBA_BWD_DKDV, s);
+      e = launch_moba_bwd_dkdv_sm100(*p, head_dim, s);
+    }
+    if (e == cudaSuccess) {
+      for (int i = 0; i < nt; ++i) p->s.order[i] = by_query[i];
+      LaunchScope scope(KVCR_K_MOBA_BWD_DQ, s);
+      e = launch_moba_bwd_dq_sm100(*p, head_dim, s);
+    }
+  }
+  delete p;
+  if (e != cudaSuccess) return cuda_fail(e, "moba_attention_bwd: launch");
+  return KVCR_OK;
+}
+
 // ===================================================================== status
 int kvcr_check_status(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int a = 0, b = 0;
+  int a = 0, b = 0, c = 0;
   cudaError_t e = read_and_clear_status_attn(&a, s);
   if (e == cudaSuccess) e = read_and_clear_status_f32(&b, s);
+  if (e == cudaSuccess) e = read_and_clear_status_bwd(&c, s);
   if (e != cudaSuccess) return cuda_fail(e, "kvcr_check_status");
-  if (a != 0 || b != 0) return fail(KVCR_ETIMEOUT, "a kernel gave up on a bounded wait");
+  if (a != 0 || b != 0 || c != 0) return fail(KVCR_ETIMEOUT, "a kernel gave up on a bounded wait");
   return KVCR_OK;
 }
 

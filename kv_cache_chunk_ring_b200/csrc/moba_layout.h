@@ -115,4 +115,49 @@ KVCR_HD void moba_row_bounds(const MobaLay& l, int r0, int r1, int& lo, int& hi)
   }
 }
 
+// Query intervals that may read the key at kpos (at most two): a key of C_j is
+// read by C_i for i >= j and by N_i for i > j; a key of N_j by N_j; a key of B
+// by B.  Returns the count; unused entries are empty ([0, 0)).
+KVCR_HD int moba_col_intervals(const MobaLay& l, int kpos, int* lo, int* hi) {
+  int kk, ki, ks, ke;
+  const int nc = l.n * l.c;
+  moba_block(l, kpos, kk, ki, ks, ke);
+  lo[0] = hi[0] = lo[1] = hi[1] = 0;
+  if (kk == kBlkC) {
+    lo[0] = ki * l.c;
+    hi[0] = nc;
+    if (ki + 1 < l.n) {
+      lo[1] = nc + (ki + 1) * l.c;
+      hi[1] = 2 * nc;
+      return 2;
+    }
+    return 1;
+  }
+  if (kk == kBlkN) {
+    lo[0] = ks;
+    hi[0] = ke;
+    return 1;
+  }
+  lo[0] = 2 * nc;
+  hi[0] = l.L;
+  return 1;
+}
+
+// Smallest query range [lo, hi) holding every query that may read a key of
+// [c0, c1).
+KVCR_HD void moba_col_bounds(const MobaLay& l, int c0, int c1, int& lo, int& hi) {
+  int kk, ki, ks, ke;
+  lo = l.L;
+  hi = 0;
+  for (int cp = c0; cp < c1; cp = ke) {
+    moba_block(l, cp, kk, ki, ks, ke);
+    int a[2], b[2];
+    const int n = moba_col_intervals(l, cp, a, b);
+    for (int t = 0; t < n; ++t) {
+      if (a[t] < lo) lo = a[t];
+      if (b[t] > hi) hi = b[t];
+    }
+  }
+}
+
 }  // namespace kvcr

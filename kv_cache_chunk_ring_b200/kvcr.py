@@ -22,17 +22,20 @@ KVCR_ECUDA, KVCR_ETIMEOUT, KVCR_ESTORAGE, KVCR_EUNSUPPORTED = -4, -5, -6, -7
 KVCR_BF16, KVCR_F32 = 0, 1
 KVCR_TILE_EMPTY, KVCR_TILE_PARTIAL, KVCR_TILE_FULL = 0, 1, 2
 (KVCR_K_APPEND_ROPE, KVCR_K_ROPE_STAGE, KVCR_K_CHUNK_ATTN, KVCR_K_MOBA_ATTN,
- KVCR_K_ATTN_F32) = range(5)
+ KVCR_K_ATTN_F32, KVCR_K_MOBA_BWD_PREP, KVCR_K_MOBA_BWD_DKDV, KVCR_K_MOBA_BWD_DQ) = range(8)
 KERNEL_NAMES = {KVCR_K_APPEND_ROPE: "append_rope", KVCR_K_ROPE_STAGE: "rope_stage",
                 KVCR_K_CHUNK_ATTN: "chunk_attn", KVCR_K_MOBA_ATTN: "moba_attn",
-                KVCR_K_ATTN_F32: "attn_f32"}
+                KVCR_K_ATTN_F32: "attn_f32", KVCR_K_MOBA_BWD_PREP: "moba_bwd_prep",
+                KVCR_K_MOBA_BWD_DKDV: "moba_bwd_dkdv", KVCR_K_MOBA_BWD_DQ: "moba_bwd_dq"}
 
 # every symbol include/kvcr.h declares
 EXPORTS = [
     "kv_cache_storage_bytes", "kv_cache_init", "kv_cache_append_rope", "kv_cache_evict",
     "kv_cache_slot_map", "kv_cache_last_append", "kv_cache_num_cached", "kv_cache_slot_data",
     "kv_cache_destroy",
-    "chunk_attention_fwd", "chunk_attention_fwd_static_scratch", "moba_attention_fwd", "moba_classify_tiles", "kvcr_check_status",
+    "chunk_attention_fwd", "chunk_attention_fwd_static_scratch", "moba_attention_fwd",
+    "moba_attention_bwd", "moba_attention_bwd_workspace_bytes", "moba_classify_tiles",
+    "kvcr_check_status",
     "kvcr_last_error", "kvcr_launch_count", "kvcr_debug_inject", "kvcr_trace_enable",
     "kvcr_trace_reset", "kvcr_trace_read",
 ]
@@ -85,6 +88,10 @@ def lib() -> ctypes.CDLL:
                                                        c_f, c_p, c_p, c_p]),
         "moba_attention_fwd": (c_int, [c_p, c_p, c_p, ctypes.POINTER(kvcr_moba_layout), c_int,
                                        c_int, c_int, c_f, c_p, c_p, c_p]),
+        "moba_attention_bwd": (c_int, [c_p, c_p, c_p, c_p, c_p, c_p,
+                                       ctypes.POINTER(kvcr_moba_layout), c_int, c_int, c_int, c_f,
+                                       c_p, c_p, c_p, c_p, c_sz, c_p]),
+        "moba_attention_bwd_workspace_bytes": (c_sz, [ctypes.POINTER(kvcr_moba_layout), c_int]),
         "moba_classify_tiles": (c_int, [ctypes.POINTER(kvcr_moba_layout), c_int, c_p, c_sz]),
         "kvcr_check_status": (c_int, [c_p]),
         "kvcr_last_error": (ctypes.c_char_p, []),
@@ -224,6 +231,30 @@ def moba_attention_fwd(q, k, v, n_chunks: int, chunk_tokens: int, n_bidir_chunks
     _check(lib().moba_attention_fwd(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(lay), q.shape[1],
                                     q.shape[2], _dtype_code(q.dtype), float(softmax_scale),
                                     _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def moba_attention_bwd_workspace_bytes(n_chunks: int, chunk_tokens: int, n_bidir_chunks: int,
+                                       heads: int) -> int:
+    lay = kvcr_moba_layout(n_chunks, chunk_tokens, n_bidir_chunks)
+    return int(lib().moba_attention_bwd_workspace_bytes(ctypes.byref(lay), heads))
+
+
+def moba_attention_bwd(q, k, v, o, d_o, lse, n_chunks: int, chunk_tokens: int,
+                       n_bidir_chunks: int, dq, dk, dv, workspace=None,
+                       softmax_scale: float = 0.0, stream=None) -> None:
+    """dQ, dK, dV of moba_attention_fwd into dq, dk, dv.  ``workspace`` is a device
+    tensor of at least moba_attention_bwd_workspace_bytes() bytes (allocated here
+    with torch when omitted)."""
+    lay = kvcr_moba_layout(n_chunks, chunk_tokens, n_bidir_chunks)
+    need = int(lib().moba_attention_bwd_workspace_bytes(ctypes.byref(lay), q.shape[1]))
+    if workspace is None:
+        import torch
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().moba_attention_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), ctypes.byref(lay),
+        q.shape[1], q.shape[2], _dtype_code(q.dtype), float(softmax_scale), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(workspace), nbytes, _stream(stream)))
 
 
 def moba_classify_tiles(n_chunks: int, chunk_tokens: int, n_bidir_chunks: int, tile: int = 128):

@@ -227,6 +227,13 @@ def moba_inputs(spec: MobaSpec) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
             draw(rng, shape, spec.dtype))
 
 
+def moba_grad_output(spec: MobaSpec) -> np.ndarray:
+    """Upstream gradient dO ([L, H, D]) for the MoBA backward: N(0, 1) in the
+    spec's dtype, from a stream of its own (the seed's PCG64 jumped once)."""
+    rng = np.random.Generator(np.random.PCG64(spec.seed).jumped(1))
+    return draw(rng, (spec.seq_len, spec.heads, spec.head_dim), spec.dtype)
+
+
 def sample_rows(n_rows: int, n_sample: int, seed: int, always: Optional[List[int]] = None) -> np.ndarray:
     """Sorted unique row indices: ``n_sample`` seeded random rows plus ``always``."""
     rng = np.random.Generator(np.random.PCG64(seed))

@@ -26,7 +26,7 @@ from typing import Iterable, Tuple
 
 import numpy as np
 
-from .moba import MobaLayout, moba_allowed
+from .moba import MobaLayout, block_of, moba_allowed
 
 
 def attention_bwd_masked(q, k, v, do, allowed: np.ndarray, scale: float
@@ -60,51 +60,65 @@ def moba_bwd_dense(q, k, v, do, lay: MobaLayout, scale: float):
     return attention_bwd_masked(q, k, v, do, moba_allowed(pos[:, None], pos[None, :], lay), scale)
 
 
-def _row_probs(q, k, lay, rows, h, scale):
-    """P rows (over all keys; zeros where not allowed) of the listed query rows, head h."""
+def _by_query_block(rows: np.ndarray, lay: MobaLayout):
+    """Yield (positions into ``rows``, sorted key indices the block may read) for
+    each query block the rows fall in; the rule is constant on a block, so its
+    first row's allowed keys are every row's."""
+    kind, idx = block_of(rows, lay)
     kpos = np.arange(lay.seq_len)
-    out = np.zeros((len(rows), lay.seq_len))
-    for n, r in enumerate(rows):
-        keys = np.nonzero(moba_allowed(r, kpos, lay))[0]
-        z = scale * (k[keys, h] @ q[r, h])
-        z = z - z.max()
-        e = np.exp(z)
-        out[n, keys] = e / e.sum()
+    for kd, ix in sorted(set(zip(kind.tolist(), idx.tolist()))):
+        sel = np.nonzero((kind == kd) & (idx == ix))[0]
+        keys = np.nonzero(moba_allowed(rows[sel[0]], kpos, lay))[0]
+        yield sel, keys
+
+
+def _rows_bwd(q, k, v, do, rows, keys, h, scale):
+    """P, dS of the given query rows over their readable keys (head h)."""
+    z = scale * (q[rows, h] @ k[keys, h].T)
+    z = z - z.max(axis=1, keepdims=True)
+    e = np.exp(z)
+    p = e / e.sum(axis=1, keepdims=True)
+    o = p @ v[keys, h]
+    dp = do[rows, h] @ v[keys, h].T
+    d = (do[rows, h] * o).sum(axis=1, keepdims=True)
+    return p, p * (dp - d)
+
+
+def moba_dq_rows(q, k, v, do, lay: MobaLayout, rows: Iterable[int], scale: float,
+                 batch: int = 1024) -> np.ndarray:
+    """dQ of the listed query rows ([n, H, D]), each from its own row of P (taken
+    over the keys the row may read; every other entry of P is zero)."""
+    q, k, v, do = (np.asarray(x, np.float64) for x in (q, k, v, do))
+    rows = np.asarray(list(rows), dtype=np.int64)
+    out = np.zeros((rows.size, q.shape[1], q.shape[2]))
+    for sel, keys in _by_query_block(rows, lay):
+        for b in range(0, sel.size, batch):
+            part = sel[b:b + batch]
+            for h in range(q.shape[1]):
+                _, ds = _rows_bwd(q, k, v, do, rows[part], keys, h, scale)
+                out[part, h] = scale * ds @ k[keys, h]
     return out
 
 
-def moba_dq_rows(q, k, v, do, lay: MobaLayout, rows: Iterable[int], scale: float) -> np.ndarray:
-    """dQ of the listed query rows ([n, H, D]), each from its own row of P."""
+def moba_dkdv_keys(q, k, v, do, lay: MobaLayout, keys: Iterable[int], scale: float,
+                   batch: int = 1024):
+    """dK and dV of the listed key rows ([n, H, D] each): the sums over every query
+    that may read them.  Each such query's row of P is evaluated in full, so pick
+    keys read by few queries."""
     q, k, v, do = (np.asarray(x, np.float64) for x in (q, k, v, do))
-    rows = list(rows)
-    H = q.shape[1]
-    out = np.zeros((len(rows), H, q.shape[2]))
-    for h in range(H):
-        p = _row_probs(q, k, lay, rows, h, scale)            # [n, L]
-        o = p @ v[:, h]
-        dp = do[rows, h] @ v[:, h].T
-        d = (do[rows, h] * o).sum(axis=1, keepdims=True)
-        ds = p * (dp - d)
-        out[:, h] = scale * ds @ k[:, h]
-    return out
-
-
-def moba_dkdv_keys(q, k, v, do, lay: MobaLayout, keys: Iterable[int], scale: float):
-    """dK and dV of the listed key rows ([n, H, D] each).  Every query that may read
-    one of the keys is evaluated in full, so pick keys read by few queries."""
-    q, k, v, do = (np.asarray(x, np.float64) for x in (q, k, v, do))
-    keys = np.asarray(list(keys))
+    keys = np.asarray(list(keys), dtype=np.int64)
     qpos = np.arange(lay.seq_len)
     readers = np.nonzero(np.any(moba_allowed(qpos[:, None], keys[None, :], lay), axis=1))[0]
     H = q.shape[1]
     dk = np.zeros((keys.size, H, q.shape[2]))
     dv = np.zeros_like(dk)
-    for h in range(H):
-        p = _row_probs(q, k, lay, readers, h, scale)          # [nq, L]
-        o = p @ v[:, h]
-        dp = do[readers, h] @ v[:, h].T
-        d = (do[readers, h] * o).sum(axis=1, keepdims=True)
-        ds = p * (dp - d)
-        dv[:, h] = p[:, keys].T @ do[readers, h]
-        dk[:, h] = scale * ds[:, keys].T @ q[readers, h]
+    for sel, ks in _by_query_block(readers, lay):
+        col = np.searchsorted(ks, keys)
+        hit = (col < ks.size) & (ks[np.minimum(col, ks.size - 1)] == keys)
+        for b in range(0, sel.size, batch):
+            r = readers[sel[b:b + batch]]
+            for h in range(H):
+                p, ds = _rows_bwd(q, k, v, do, r, ks, h, scale)
+                dv[hit, h] += p[:, col[hit]].T @ do[r, h]
+                dk[hit, h] += scale * ds[:, col[hit]].T @ q[r, h]
     return dk, dv

@@ -155,3 +155,31 @@ def test_classify_tiles_full_size_matches_oracle():
     ref = classify_tiles_blocks(MobaLayout(spec.n_chunks, spec.chunk_tokens, spec.n_bidir_chunks), 128)
     assert got.shape == (1131, 1131)
     assert np.array_equal(got, ref)
+
+
+def test_moba_bwd_workspace_bytes():
+    # 8 bytes per (head, row), rows rounded up to a multiple of 128
+    assert kvcr.moba_attention_bwd_workspace_bytes(2, 200, 1, 3) == 3 * 1024 * 8   # L = 1000
+    assert kvcr.moba_attention_bwd_workspace_bytes(8, 6032, 8, 12) == 12 * 1131 * 128 * 8
+    assert kvcr.moba_attention_bwd_workspace_bytes(0, 200, 1, 3) == 0
+    assert kvcr.moba_attention_bwd_workspace_bytes(2, 200, 1, 0) == 0
+
+
+def test_moba_bwd_rejects_bad_arguments_before_launch():
+    import ctypes
+    L = kvcr.lib()
+    lay = kvcr.kvcr_moba_layout(2, 200, 1)
+    p = ctypes.c_void_p(1 << 20)                     # aligned, never dereferenced
+    args = lambda **kw: [kw.get(n, p) for n in ("q", "k", "v", "o", "do", "lse")]
+    call = lambda *a, dtype=kvcr.KVCR_BF16, hd=128, ws_bytes=1 << 30, ws=p, dq=p: \
+        L.moba_attention_bwd(*a, ctypes.byref(lay), 2, hd, dtype, 0.0, dq, p, p, ws, ws_bytes,
+                             None)
+    assert call(*args(), dtype=kvcr.KVCR_F32) == kvcr.KVCR_EUNSUPPORTED
+    assert call(*args(), hd=96) == kvcr.KVCR_EUNSUPPORTED
+    assert call(*args(q=None)) == kvcr.KVCR_EINVAL
+    assert call(*args(), dq=None) == kvcr.KVCR_EINVAL
+    assert call(*args(k=ctypes.c_void_p((1 << 20) + 8))) == kvcr.KVCR_EINVAL
+    assert call(*args(), ws_bytes=16) == kvcr.KVCR_ESTORAGE
+    bad = kvcr.kvcr_moba_layout(0, 200, 1)
+    assert L.moba_attention_bwd(p, p, p, p, p, p, ctypes.byref(bad), 2, 128, kvcr.KVCR_BF16, 0.0,
+                                p, p, p, p, 1 << 30, None) == kvcr.KVCR_ESHAPE
