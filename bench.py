@@ -19,6 +19,7 @@ workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -553,6 +554,67 @@ def run_moba(args) -> dict:
             "steps": args.steps, "warmup": args.warmup}
 
 
+def run_moba_bwd(args) -> dict:
+    """MoBA backward (dQ, dK, dV) over the 144768-token training sequence, from the
+    forward's O and LSE; also the forward + backward step."""
+    import torch
+    from kv_cache_chunk_ring_b200 import build as _build
+    from kv_cache_chunk_ring_b200 import kvcr
+    _build.build()
+    spec = wl.MOBA_8x6032
+    if args.moba_chunk_tokens:                        # a smaller sequence of the same shape
+        spec = dataclasses.replace(spec, name=f"moba_8chunks_x{args.moba_chunk_tokens}",
+                                   chunk_tokens=args.moba_chunk_tokens)
+    lay = (spec.n_chunks, spec.chunk_tokens, spec.n_bidir_chunks)
+    gen = torch.Generator(device="cuda").manual_seed(spec.seed)
+    shape = (spec.seq_len, spec.heads, spec.head_dim)
+    q, k, v, do = (_randn(shape, gen) for _ in range(4))
+    o = torch.empty_like(q)
+    lse = torch.empty((spec.heads, spec.seq_len), dtype=torch.float32, device="cuda")
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = torch.empty(kvcr.moba_attention_bwd_workspace_bytes(*lay, spec.heads), dtype=torch.uint8,
+                     device="cuda")
+    kvcr.moba_attention_fwd(q, k, v, *lay, o, lse)
+
+    def bwd():
+        kvcr.moba_attention_bwd(q, k, v, o, do, lse, *lay, dq, dk, dv, workspace=ws)
+
+    def fwd_bwd():
+        kvcr.moba_attention_fwd(q, k, v, *lay, o, lse)
+        bwd()
+
+    ms = _timed(bwd, args.steps, args.warmup)
+    ms_step = _timed(fwd_bwd, max(2, args.steps // 2), 1)
+    kvcr.kvcr_check_status()
+    kvcr.kvcr_trace_reset()
+    kvcr.kvcr_trace_enable(True)
+    bwd()
+    torch.cuda.synchronize()
+    kvcr.kvcr_trace_enable(False)
+    kt = {name: kvcr.kvcr_trace_read(kid) for kid, name in kvcr.KERNEL_NAMES.items()}
+    kvcr.kvcr_trace_reset()
+    fwd_flops = moba_useful_flops(spec)
+    flops = 2.5 * fwd_flops          # dV, dP, dQ, dK and the recomputed S: five products
+    peaks, kind = load_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+
+    def kms(name):
+        n, t = kt[name]
+        return t / max(1, n)
+    dkdv_ms, dq_ms = kms("moba_bwd_dkdv"), kms("moba_bwd_dq")
+    return {"workload": spec.name + "_backward", "ms_per_call": round(ms, 3),
+            "useful_tflop": round(flops / 1e12, 3), "value": round(tf, 2), "unit": UNIT,
+            "frac_of_peak": round(tf / peaks["bf16_tflops"], 4),
+            "kernels_ms": {"prep": round(kms("moba_bwd_prep"), 4), "dkdv": round(dkdv_ms, 3),
+                           "dq": round(dq_ms, 3)},
+            # executed tensor work: dK/dV kernel 4 products, dQ kernel 3 (S and dP recomputed)
+            "executed_tflops": {"dkdv": round(2.0 * fwd_flops / (dkdv_ms * 1e-3) / 1e12, 1),
+                                "dq": round(1.5 * fwd_flops / (dq_ms * 1e-3) / 1e12, 1)},
+            "fwd_bwd_ms": round(ms_step, 3),
+            "fwd_bwd_tflops": round(3.5 * fwd_flops / (ms_step * 1e-3) / 1e12, 2),
+            "steps": args.steps, "warmup": args.warmup}
+
+
 def run_dynwin(args) -> dict:
     """720p rollout, 6 anchors, window drawn per chunk from U{2..8}, plus cross-attention."""
     import torch
@@ -615,7 +677,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="chunk", choices=["chunk", "layers30", "moba", "dynwin"],
+    ap.add_argument("--moba-chunk-tokens", type=int, default=0,
+                    help="moba_bwd: tokens per chunk (default: the workload's 6032); a smaller "
+                         "value gives a case small enough for a full profiler capture")
+    ap.add_argument("--workload", default="chunk", choices=["chunk", "layers30", "moba", "moba_bwd", "dynwin"],
                     help="chunk: the 832x464 steady-state step (the bench line); the others "
                          "print single-GPU timings of the other workloads")
     args = ap.parse_args()
@@ -629,7 +694,8 @@ def main():
             print(json.dumps(run_reference(args)))
         return
     if args.workload != "chunk":
-        fn = {"layers30": run_layers30, "moba": run_moba, "dynwin": run_dynwin}[args.workload]
+        fn = {"layers30": run_layers30, "moba": run_moba, "moba_bwd": run_moba_bwd,
+              "dynwin": run_dynwin}[args.workload]
         if rank == 0:
             print(json.dumps(fn(args)))
         return
