@@ -19,7 +19,7 @@ struct MobaBwdParams {
   CUtensorMap tm_k;
   CUtensorMap tm_v;
   CUtensorMap tm_do;
-  const float2* ws;    // [H][Lpad] (lse * log2 e, rowsum(dO o O)); Lpad = 128 * n_units
+  const float* ws;     // [H][n_units][2][128]: lse * log2 e, then rowsum(dO o O), of a tile's rows
   void* dq;            // [L][H][D] bf16
   void* dk;
   void* dv;
@@ -36,7 +36,7 @@ struct MobaBwdPrepParams {
   const void* o;       // [L][H][D] bf16
   const void* d_o;
   const float* lse;    // [H][L], natural log
-  float2* ws;          // [H][Lpad]
+  float* ws;           // [H][Lpad / 128][2][128]
   int L, Lpad, H;
 };
 

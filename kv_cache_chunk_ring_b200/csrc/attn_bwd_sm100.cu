@@ -11,7 +11,8 @@
 // in fp32 on the tensor cores (bf16 operands), written back as bf16.
 //
 // Three launches, no atomics (the result does not depend on scheduling):
-//   prep   ws[h][i] = (LSE_i * log2 e, D_i); rows past L get (+inf, 0), so
+//   prep   per head and 128-row tile: LSE_i * log2 e of its rows, then D_i of
+//          them (ws[h][t][0][r], ws[h][t][1][r]); rows past L get (+inf, 0), so
 //          their probabilities are exactly 0.
 //   dK/dV  one CTA per (head, 128-key tile); K_j, V_j stay in shared memory and
 //          the query tiles that may read them stream through a 2-stage ring:
@@ -266,7 +267,7 @@ __device__ void bwd_producer(const MobaBwdParams& p, BwdCtl* ctl, uint8_t* smem,
     load_tile<HD>(sx, smem + L::kX + st * L::kTileBytes, &ctl->st_full[st], h, u * kTile);
     load_tile<HD>(sy, smem + L::kY + st * L::kTileBytes, &ctl->st_full[st], h, u * kTile);
     if (kByKey)
-      bulk_load(smem + L::kW + st * kWsBytes, p.ws + (size_t)h * p.Lpad + (size_t)u * kTile,
+      bulk_load(smem + L::kW + st * kWsBytes, p.ws + ((size_t)h * p.s.n_units + u) * 2 * kTile,
                 kWsBytes, &ctl->st_full[st]);
     issued = i + 1;
   }
@@ -404,8 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
       tmem_ld_32x32b_x32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_ld_32x32b_x32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
       tmem_ld_wait();
-      // (lse * log2 e, D) of columns 2e and 2e + 1 of this warpgroup
-      const float4* w4 = reinterpret_cast<const float4*>(smem + L::kW + st * kWsBytes) + wg * 32;
+      // lse * log2 e (l4) and D (d4) of columns 4m .. 4m + 3 of this warpgroup
+      const float4* l4 = reinterpret_cast<const float4*>(smem + L::kW + st * kWsBytes) + wg * 16;
+      const float4* d4 = l4 + kTile / 4;
       uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
       if (cls != kTileFull) {
 #pragma unroll
@@ -422,9 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const int n = 32 * c + 2 * q;
-          const float4 wv = w4[n >> 1];
+          const float4 lv = l4[n >> 2];
           const float2 x = ffma2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])),
-                                 sl2x2, make_float2(-wv.x, -wv.z));
+                                 sl2x2, (q & 1) ? make_float2(-lv.z, -lv.w)
+                                                : make_float2(-lv.x, -lv.y));
           float p0 = ex2_sfu(x.x), p1 = ex2_sfu(x.y);
           if (!((keep[c] >> (2 * q)) & 1u)) p0 = 0.f;
           if (!((keep[c] >> (2 * q + 1)) & 1u)) p1 = 0.f;
@@ -454,9 +457,9 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const int n = 32 * c + 2 * q;
-          const float4 wv = w4[n >> 1];
-          const float d0 = pr[n] * (__uint_as_float(s[n]) - wv.y);
-          const float d1 = pr[n + 1] * (__uint_as_float(s[n + 1]) - wv.w);
+          const float4 dv = d4[n >> 2];
+          const float d0 = pr[n] * (__uint_as_float(s[n]) - ((q & 1) ? dv.z : dv.x));
+          const float d1 = pr[n + 1] * (__uint_as_float(s[n + 1]) - ((q & 1) ? dv.w : dv.y));
           packed[q] = pack_bf16(d0, d1);
         }
         tmem_st_32x32b_x16(dp_addr + c * 16, packed);
@@ -584,7 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
     const uint32_t dp_addr = tmem + lane_base + kTmemDP + (uint32_t)wg * 64u;
     const float sl2 = p.scale_log2;
     const MobaLay lay{p.s.n_chunks, p.s.chunk_tokens, p.s.n_bidir, p.s.L};
-    const float2 wrow = p.ws[(size_t)h * p.Lpad + q0 + r];
+    const float* wt = p.ws + ((size_t)h * p.s.n_units + qt) * 2 * kTile;
+    const float2 wrow = make_float2(wt[r], wt[kTile + r]);   // (lse * log2 e, D) of row q0 + r
     const float2 sl2x2 = make_float2(sl2, sl2);
     const float2 neg_lse = make_float2(-wrow.x, -wrow.x);
     int a[2] = {0, 0}, b[2] = {0, 0};
@@ -735,7 +739,9 @@ __global__ void __launch_bounds__(256) moba_bwd_prep_kernel(const MobaBwdPrepPar
       const float v = p.lse[(size_t)h * p.L + row];
       if (v != -INFINITY) lse2 = v * 1.4426950408889634f;
     }
-    p.ws[item] = make_float2(lse2, live ? acc : 0.f);
+    float* wt = p.ws + ((size_t)h * (p.Lpad / kTile) + row / kTile) * 2 * kTile;
+    wt[row % kTile] = lse2;
+    wt[kTile + row % kTile] = live ? acc : 0.f;
   }
 }
 

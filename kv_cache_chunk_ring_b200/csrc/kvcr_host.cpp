@@ -957,7 +957,7 @@ size_t moba_attention_bwd_workspace_bytes(const kvcr_moba_layout* layout, int he
   MobaLay l;
   if (moba_check_layout(layout, &l) != KVCR_OK || heads < 1) return 0;
   const size_t lpad = (size_t)((l.L + kTile - 1) / kTile) * kTile;
-  return lpad * (size_t)heads * sizeof(float2);
+  return lpad * (size_t)heads * 2 * sizeof(float);
 }
 
 int moba_attention_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -1005,7 +1005,7 @@ int moba_attention_bwd(const void* q, const void* k, const void* v, const void* 
     return rc;
   }
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)head_dim);
-  float2* ws = static_cast<float2*>(workspace);
+  float* ws = static_cast<float*>(workspace);
   p->ws = ws;
   p->dq = dq;
   p->dk = dk;
