@@ -670,6 +670,65 @@ def run_dynwin(args) -> dict:
             "note": "per chunk: evict(W_t), self-attention, cross-attention (512 text keys), append"}
 
 
+def run_aux(args) -> dict:
+    """832x464 steady-state chunk step with 4 auxiliary evidence frames: per chunk,
+    kv_cache_set_aux (4 frames, K rotated at their positions), 4 denoising-step
+    attention calls over 6 + 8 cached + 4 auxiliary + 4 current frames (33176 keys),
+    append (which drops the auxiliary frames)."""
+    import torch
+    from kv_cache_chunk_ring_b200 import build as _build
+    from kv_cache_chunk_ring_b200 import kvcr
+    _build.build()
+    spec, n_aux, steps = SPEC, 4, 4
+    T, H, D, F = spec.tokens_per_frame, spec.heads, spec.head_dim, spec.chunk_frames
+    cache = kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope(), aux_frames=n_aux)
+    gen = torch.Generator(device="cuda").manual_seed(spec.seed)
+    pool = [tuple(_randn((spec.chunk_tokens, H, D), gen) for _ in range(3)) for _ in range(3)]
+    aux_k, aux_v = _randn((n_aux * T, H, D), gen), _randn((n_aux * T, H, D), gen)
+    o = torch.empty_like(pool[0][0])
+    state = {"c": 0}
+
+    def chunk():
+        c = state["c"]
+        frames = list(range(c * F, (c + 1) * F))
+        if c >= STEADY_CHUNK:
+            cache.set_aux(aux_k, aux_v, [max(0, c * F - 8 + i) for i in range(n_aux)])
+        for s in range(steps):
+            q, k, v = pool[(c + s) % 3]
+            cache.attention(q, k, v, frames, out=o)
+        cache.append(k, v, frames)
+        state["c"] = c + 1
+
+    for _ in range(STEADY_CHUNK):
+        chunk()
+    ms = _timed(chunk, args.steps, args.warmup)
+    kvcr.kvcr_trace_reset()
+    kvcr.kvcr_trace_enable(True)
+    chunk()
+    torch.cuda.synchronize()
+    kvcr.kvcr_trace_enable(False)
+    kt = {name: kvcr.kvcr_trace_read(kid) for kid, name in kvcr.KERNEL_NAMES.items()}
+    kvcr.kvcr_trace_reset()
+    kvcr.kvcr_check_status()
+    lk = (spec.sinks + spec.window + n_aux + F) * T
+    call_flops = 4.0 * spec.chunk_tokens * lk * H * D
+    attn_n, attn_ms = kt["chunk_attn"]
+    aux_n, aux_ms = kt["set_aux"]
+    peaks, kind = load_peaks()
+    attn_call = attn_ms / max(1, attn_n)
+    aux_bytes = 4.0 * n_aux * T * H * D * 2          # read and write K and V
+    return {"workload": spec.name + "_aux4", "keys_per_call": lk,
+            "ms_per_chunk": round(ms, 3), "calls_per_chunk": steps,
+            "value": round(steps * call_flops / (ms * 1e-3) / 1e12, 2), "unit": UNIT,
+            "attn_kernel_ms": round(attn_call, 4),
+            "attn_tflops": round(call_flops / (attn_call * 1e-3) / 1e12, 1),
+            "attn_frac_of_peak": round(call_flops / (attn_call * 1e-3) / 1e12 /
+                                       peaks["bf16_tflops"], 4),
+            "set_aux_us": round(1e3 * aux_ms / max(1, aux_n), 2),
+            "set_aux_gb_s": round(aux_bytes / (aux_ms / max(1, aux_n) * 1e-3) / 1e9, 1),
+            "steps": args.steps, "warmup": args.warmup}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -680,7 +739,7 @@ def main():
     ap.add_argument("--moba-chunk-tokens", type=int, default=0,
                     help="moba_bwd: tokens per chunk (default: the workload's 6032); a smaller "
                          "value gives a case small enough for a full profiler capture")
-    ap.add_argument("--workload", default="chunk", choices=["chunk", "layers30", "moba", "moba_bwd", "dynwin"],
+    ap.add_argument("--workload", default="chunk", choices=["chunk", "layers30", "moba", "moba_bwd", "dynwin", "aux"],
                     help="chunk: the 832x464 steady-state step (the bench line); the others "
                          "print single-GPU timings of the other workloads")
     args = ap.parse_args()
@@ -695,7 +754,7 @@ def main():
         return
     if args.workload != "chunk":
         fn = {"layers30": run_layers30, "moba": run_moba, "moba_bwd": run_moba_bwd,
-              "dynwin": run_dynwin}[args.workload]
+              "dynwin": run_dynwin, "aux": run_aux}[args.workload]
         if rank == 0:
             print(json.dumps(fn(args)))
         return

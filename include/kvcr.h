@@ -114,7 +114,41 @@ int kv_cache_init(kvcr_cache **out, int sinks, int window, int tokens_per_frame,
                   int head_dim, int chunk_frames, const kvcr_rope *rope, kvcr_dtype dtype,
                   void *device_storage, size_t storage_bytes);
 
-/* Append finalized frames (the last denoising step's K and V).
+/* Caches with auxiliary slots: temporary attention blocks that carry extra
+ * evidence for the current chunk and are removed once it is finalized ("Westlake
+ * AGI Lab's 'World in World' Steers Frozen Video Models", second paragraph:
+ * source-video observations, target-view projections, rendered geometry,
+ * retrieved history, read through the backbone's own attention).  aux_frames
+ * more frame slots (sinks + window + aux_frames <= 32) follow the anchor and
+ * window slots in the storage; everything else is as for kv_cache_storage_bytes()
+ * and kv_cache_init(), which are these with aux_frames = 0. */
+size_t kv_cache_storage_bytes_aux(int sinks, int window, int aux_frames, int tokens_per_frame,
+                                  int heads, int head_dim, int chunk_frames, int with_rope,
+                                  kvcr_dtype dtype);
+int kv_cache_init_aux(kvcr_cache **out, int sinks, int window, int aux_frames,
+                      int tokens_per_frame, int heads, int head_dim, int chunk_frames,
+                      const kvcr_rope *rope, kvcr_dtype dtype, void *device_storage,
+                      size_t storage_bytes);
+
+/* Write n_frames auxiliary frames for the current chunk, replacing any set
+ * before: k, v device [n_frames * tokens_per_frame][heads][head_dim].  With a
+ * RoPE cache and aux_pos != NULL (host, n_frames temporal positions >= 0, e.g. the
+ * evidence's event time), K is rotated by RoPE3D at (aux_pos[f], h, w); with
+ * aux_pos = NULL (or a cache without RoPE), K is stored as given.  V as is.
+ * Every chunk_attention_fwd*() call then reads them after the cached frames,
+ * until the next kv_cache_append_rope() (the chunk's finalization) drops them;
+ * they never enter the anchor / window slots and are never evicted.  0 <=
+ * n_frames <= aux_frames (n_frames = 0 drops them now).  Bookkeeping-only
+ * caches take k = v = NULL.  Errors: KVCR_ESHAPE (n_frames), KVCR_EINVAL (NULL or
+ * misaligned k / v, negative position), KVCR_ESTATE; nothing changes on error. */
+int kv_cache_set_aux(kvcr_cache *c, const void *k, const void *v, const int32_t *aux_pos,
+                     int n_frames, void *stream);
+
+/* Number of auxiliary frames the next attention call reads. */
+int kv_cache_num_aux(const kvcr_cache *c, int *n);
+
+/* Append finalized frames (the last denoising step's K and V); this finalizes the
+ * chunk, so its auxiliary frames (kv_cache_set_aux) are dropped.
  * k, v: device [n_frames * tokens_per_frame][heads][head_dim].  frame_idx: host,
  * n_frames strictly increasing absolute latent-frame indices, each larger than
  * every frame appended before.  Frame by frame: an unfilled anchor slot is taken
@@ -145,7 +179,8 @@ int kv_cache_last_append(const kvcr_cache *c, int32_t *slots, int slots_cap,
 int kv_cache_num_cached(const kvcr_cache *c, int *n);
 
 /* Device addresses of slot `slot`'s K and V, each [tokens_per_frame][heads][head_dim]
- * in the cache dtype (K stored rotated).  For reading back or saving a cache. */
+ * in the cache dtype (K stored rotated).  For reading back or saving a cache.
+ * Slots sinks + window .. + aux_frames - 1 are the auxiliary slots. */
 int kv_cache_slot_data(const kvcr_cache *c, int slot, const void **k, const void **v);
 
 void kv_cache_destroy(kvcr_cache *c);
@@ -266,7 +301,8 @@ enum {
     KVCR_K_MOBA_BWD_PREP = 5, /* MoBA backward: per-row LSE and rowsum(dO o O) */
     KVCR_K_MOBA_BWD_DKDV = 6, /* MoBA backward: dK and dV (tensor cores) */
     KVCR_K_MOBA_BWD_DQ = 7,   /* MoBA backward: dQ (tensor cores) */
-    KVCR_K_COUNT = 8
+    KVCR_K_SET_AUX = 8,       /* auxiliary frames written into their slots (RoPE3D of K) */
+    KVCR_K_COUNT = 9
 };
 
 /* Count of every kernel the library launched in this process. */

@@ -164,13 +164,13 @@ struct StorageLayout {
   size_t k_off, v_off, q_off, ks_off, h_off, w_off, total;
 };
 
-bool make_layout(int S, int W, int T, int H, int D, int F, bool rope, size_t esize,
+bool make_layout(int S, int W, int A, int T, int H, int D, int F, bool rope, size_t esize,
                  StorageLayout* L) {
-  if (S < 0 || W < 0 || S + W < 1 || S + W > kMaxSlots || T < 1 || H < 1 || D < 1 || F < 1 ||
-      F > kMaxFrames)
+  if (S < 0 || W < 0 || A < 0 || S + W < 1 || S + W + A > kMaxSlots || T < 1 || H < 1 || D < 1 ||
+      F < 1 || F > kMaxFrames)
     return false;
   const size_t frame = (size_t)T * H * D * esize;
-  const size_t slots = (size_t)(S + W);
+  const size_t slots = (size_t)(S + W + A);  // anchors, window, auxiliary
   size_t off = 0;
   L->k_off = off;
   off = align_up(off + slots * frame, 256);
@@ -197,6 +197,8 @@ bool make_layout(int S, int W, int T, int H, int D, int F, bool rope, size_t esi
 // ====================================================================== cache
 struct kvcr_cache {
   int S, W, T, H, D, F;
+  int A;      // auxiliary slots (physical slots S + W .. S + W + A - 1)
+  int n_aux;  // auxiliary frames visible to the current chunk's attention
   kvcr_dtype dtype;
   size_t esize;
   bool rope;
@@ -307,26 +309,43 @@ extern "C" {
 
 const char* kvcr_last_error(void) { return g_err.c_str(); }
 
-size_t kv_cache_storage_bytes(int sinks, int window, int tokens_per_frame, int heads, int head_dim,
-                              int chunk_frames, int with_rope, kvcr_dtype dtype) {
+size_t kv_cache_storage_bytes_aux(int sinks, int window, int aux_frames, int tokens_per_frame,
+                                  int heads, int head_dim, int chunk_frames, int with_rope,
+                                  kvcr_dtype dtype) {
   if (dtype != KVCR_BF16 && dtype != KVCR_F32) return 0;
   StorageLayout L;
-  if (!make_layout(sinks, window, tokens_per_frame, heads, head_dim, chunk_frames, with_rope != 0,
-                   dtype == KVCR_BF16 ? 2 : 4, &L))
+  if (!make_layout(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
+                   with_rope != 0, dtype == KVCR_BF16 ? 2 : 4, &L))
     return 0;
   return L.total;
+}
+
+size_t kv_cache_storage_bytes(int sinks, int window, int tokens_per_frame, int heads, int head_dim,
+                              int chunk_frames, int with_rope, kvcr_dtype dtype) {
+  return kv_cache_storage_bytes_aux(sinks, window, 0, tokens_per_frame, heads, head_dim,
+                                    chunk_frames, with_rope, dtype);
 }
 
 int kv_cache_init(kvcr_cache** out, int sinks, int window, int tokens_per_frame, int heads,
                   int head_dim, int chunk_frames, const kvcr_rope* rope, kvcr_dtype dtype,
                   void* device_storage, size_t storage_bytes) {
+  return kv_cache_init_aux(out, sinks, window, 0, tokens_per_frame, heads, head_dim, chunk_frames,
+                           rope, dtype, device_storage, storage_bytes);
+}
+
+int kv_cache_init_aux(kvcr_cache** out, int sinks, int window, int aux_frames,
+                      int tokens_per_frame, int heads, int head_dim, int chunk_frames,
+                      const kvcr_rope* rope, kvcr_dtype dtype, void* device_storage,
+                      size_t storage_bytes) {
   if (out == nullptr) return fail(KVCR_EINVAL, "kv_cache_init: out is NULL");
   *out = nullptr;
   if (dtype != KVCR_BF16 && dtype != KVCR_F32) return fail(KVCR_EINVAL, "kv_cache_init: bad dtype");
   if (head_dim != 64 && head_dim != 128)
     return fail(KVCR_EUNSUPPORTED, "kv_cache_init: head_dim must be 64 or 128");
-  if (sinks < 0 || window < 0 || sinks + window < 1 || sinks + window > kMaxSlots)
-    return fail(KVCR_ESHAPE, "kv_cache_init: need 1 <= sinks + window <= 32");
+  if (sinks < 0 || window < 0 || aux_frames < 0 || sinks + window < 1 ||
+      sinks + window + aux_frames > kMaxSlots)
+    return fail(KVCR_ESHAPE,
+                "kv_cache_init: need 1 <= sinks + window and sinks + window + aux_frames <= 32");
   if (tokens_per_frame < 1 || heads < 1 || chunk_frames < 1 || chunk_frames > kMaxFrames)
     return fail(KVCR_ESHAPE, "kv_cache_init: bad tokens_per_frame / heads / chunk_frames (<= 16)");
   if ((long long)chunk_frames * tokens_per_frame > (1LL << 30) ||
@@ -344,8 +363,8 @@ int kv_cache_init(kvcr_cache** out, int sinks, int window, int tokens_per_frame,
   }
   const size_t esize = dtype == KVCR_BF16 ? 2 : 4;
   StorageLayout L;
-  if (!make_layout(sinks, window, tokens_per_frame, heads, head_dim, chunk_frames, rope != nullptr,
-                   esize, &L))
+  if (!make_layout(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
+                   rope != nullptr, esize, &L))
     return fail(KVCR_ESHAPE, "kv_cache_init: bad sizes");
   const bool has_storage = device_storage != nullptr;
   if (!has_storage && storage_bytes != 0)
@@ -364,6 +383,8 @@ int kv_cache_init(kvcr_cache** out, int sinks, int window, int tokens_per_frame,
   kvcr_cache* c = new kvcr_cache();
   c->S = sinks;
   c->W = window;
+  c->A = aux_frames;
+  c->n_aux = 0;
   c->T = tokens_per_frame;
   c->H = heads;
   c->D = head_dim;
@@ -407,7 +428,7 @@ int kv_cache_init(kvcr_cache** out, int sinks, int window, int tokens_per_frame,
     }
     if (dtype == KVCR_BF16) {
       const uint64_t dims[4] = {(uint64_t)head_dim, (uint64_t)heads, (uint64_t)tokens_per_frame,
-                                (uint64_t)(sinks + window)};
+                                (uint64_t)(sinks + window + aux_frames)};
       int rc = encode_bf16_map(&c->tm_kc, c->storage + L.k_off, 4, dims, kKeyTile);
       if (!rc) rc = encode_bf16_map(&c->tm_vc, c->storage + L.v_off, 4, dims, kKeyTile);
       if (rc) {
@@ -430,6 +451,7 @@ int kv_cache_append_rope(kvcr_cache* c, const void* k, const void* v, const int3
   if (n_frames == 0) {
     c->last_slots.clear();
     c->last_evicted.clear();
+    c->n_aux = 0;
     return KVCR_OK;
   }
   int rc = check_frames(c, frame_idx, n_frames, "kv_cache_append_rope");
@@ -480,6 +502,7 @@ int kv_cache_append_rope(kvcr_cache* c, const void* k, const void* v, const int3
   }
   c->last_slots = slots;
   c->last_evicted = evicted;
+  c->n_aux = 0;  // the chunk is finalized: its auxiliary frames are dropped
   return KVCR_OK;
 }
 
@@ -532,10 +555,62 @@ int kv_cache_slot_data(const kvcr_cache* c, int slot, const void** k, const void
   if (c == nullptr || k == nullptr || v == nullptr)
     return fail(KVCR_EINVAL, "kv_cache_slot_data: NULL");
   if (!c->has_storage) return fail(KVCR_ESTATE, "kv_cache_slot_data: bookkeeping-only cache");
-  if (slot < 0 || slot >= c->S + c->W) return fail(KVCR_EINVAL, "kv_cache_slot_data: bad slot");
+  if (slot < 0 || slot >= c->S + c->W + c->A)
+    return fail(KVCR_EINVAL, "kv_cache_slot_data: bad slot");
   const size_t frame = (size_t)c->T * c->H * c->D * c->esize;
   *k = c->storage + c->lay.k_off + (size_t)slot * frame;
   *v = c->storage + c->lay.v_off + (size_t)slot * frame;
+  return KVCR_OK;
+}
+
+int kv_cache_set_aux(kvcr_cache* c, const void* k, const void* v, const int32_t* aux_pos,
+                     int n_frames, void* stream) {
+  const char* fn = "kv_cache_set_aux";
+  if (c == nullptr) return fail(KVCR_EINVAL, std::string(fn) + ": cache is NULL");
+  if (n_frames < 0 || n_frames > c->A || n_frames > kMaxFrames)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_frames must be in [0, aux_frames] (<= 16)");
+  if (aux_pos != nullptr)
+    for (int i = 0; i < n_frames; ++i)
+      if (aux_pos[i] < 0) return fail(KVCR_EINVAL, std::string(fn) + ": negative position");
+  if (c->has_storage && n_frames > 0) {
+    if (k == nullptr || v == nullptr) return fail(KVCR_EINVAL, std::string(fn) + ": k/v NULL");
+    if (!aligned16(k) || !aligned16(v))
+      return fail(KVCR_EINVAL, std::string(fn) + ": k/v must be 16-byte aligned");
+  } else if (!c->has_storage && (k != nullptr || v != nullptr)) {
+    return fail(KVCR_ESTATE, std::string(fn) + ": bookkeeping-only cache takes k = v = NULL");
+  }
+  if (c->has_storage && n_frames > 0) {
+    RopeCopyParams p;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(c, p);
+    p.src_a = k;
+    p.src_b = v;
+    p.dst_a = c->storage + c->lay.k_off;
+    p.dst_b = c->storage + c->lay.v_off;
+    p.rotate_a = (c->rope && aux_pos != nullptr) ? 1 : 0;
+    p.rotate_b = 0;
+    p.n_frames = n_frames;
+    const long long frame_elems = (long long)c->T * c->H * c->D;
+    for (int f = 0; f < n_frames; ++f) {
+      p.dst_frame_off[f] = (long long)(c->S + c->W + f) * frame_elems;
+      p.src_frame[f] = f;
+    }
+    if (p.rotate_a) fill_ttab(c, p, aux_pos, n_frames);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    {
+      LaunchScope scope(KVCR_K_SET_AUX, s);
+      e = launch_rope_copy(p, c->dtype, s, c->n_sm);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "kv_cache_set_aux: launch");
+  }
+  c->n_aux = n_frames;
+  return KVCR_OK;
+}
+
+int kv_cache_num_aux(const kvcr_cache* c, int* n) {
+  if (c == nullptr || n == nullptr) return fail(KVCR_EINVAL, "kv_cache_num_aux: NULL");
+  *n = c->n_aux;
   return KVCR_OK;
 }
 
@@ -568,6 +643,7 @@ int chunk_attention_fwd(kvcr_cache* c, const void* q, int n_q, const void* k_cur
   int n_vis = 0;
   for (int i = 0; i < c->S + c->W; ++i)
     if (c->slot_frame[i] >= 0) slots[n_vis++] = i;
+  for (int i = 0; i < c->n_aux; ++i) slots[n_vis++] = c->S + c->W + i;  // auxiliary frames
 
   const void* q_src = q;
   const void* k_src = k_cur;
@@ -698,6 +774,7 @@ int chunk_attention_fwd_static_scratch(kvcr_cache* c, const void* q, int n_q, co
   int n_vis = 0;
   for (int i = 0; i < c->S + c->W; ++i)
     if (c->slot_frame[i] >= 0) slots[n_vis++] = i;
+  for (int i = 0; i < c->n_aux; ++i) slots[n_vis++] = c->S + c->W + i;  // auxiliary frames
 
   const void* q_src = q;
   const void* k_src = k_cur;

@@ -22,15 +22,18 @@ KVCR_ECUDA, KVCR_ETIMEOUT, KVCR_ESTORAGE, KVCR_EUNSUPPORTED = -4, -5, -6, -7
 KVCR_BF16, KVCR_F32 = 0, 1
 KVCR_TILE_EMPTY, KVCR_TILE_PARTIAL, KVCR_TILE_FULL = 0, 1, 2
 (KVCR_K_APPEND_ROPE, KVCR_K_ROPE_STAGE, KVCR_K_CHUNK_ATTN, KVCR_K_MOBA_ATTN,
- KVCR_K_ATTN_F32, KVCR_K_MOBA_BWD_PREP, KVCR_K_MOBA_BWD_DKDV, KVCR_K_MOBA_BWD_DQ) = range(8)
+ KVCR_K_ATTN_F32, KVCR_K_MOBA_BWD_PREP, KVCR_K_MOBA_BWD_DKDV, KVCR_K_MOBA_BWD_DQ,
+ KVCR_K_SET_AUX) = range(9)
 KERNEL_NAMES = {KVCR_K_APPEND_ROPE: "append_rope", KVCR_K_ROPE_STAGE: "rope_stage",
                 KVCR_K_CHUNK_ATTN: "chunk_attn", KVCR_K_MOBA_ATTN: "moba_attn",
                 KVCR_K_ATTN_F32: "attn_f32", KVCR_K_MOBA_BWD_PREP: "moba_bwd_prep",
-                KVCR_K_MOBA_BWD_DKDV: "moba_bwd_dkdv", KVCR_K_MOBA_BWD_DQ: "moba_bwd_dq"}
+                KVCR_K_MOBA_BWD_DKDV: "moba_bwd_dkdv", KVCR_K_MOBA_BWD_DQ: "moba_bwd_dq",
+                KVCR_K_SET_AUX: "set_aux"}
 
 # every symbol include/kvcr.h declares
 EXPORTS = [
-    "kv_cache_storage_bytes", "kv_cache_init", "kv_cache_append_rope", "kv_cache_evict",
+    "kv_cache_storage_bytes", "kv_cache_init", "kv_cache_storage_bytes_aux", "kv_cache_init_aux",
+    "kv_cache_set_aux", "kv_cache_num_aux", "kv_cache_append_rope", "kv_cache_evict",
     "kv_cache_slot_map", "kv_cache_last_append", "kv_cache_num_cached", "kv_cache_slot_data",
     "kv_cache_destroy",
     "chunk_attention_fwd", "chunk_attention_fwd_static_scratch", "moba_attention_fwd",
@@ -75,6 +78,11 @@ def lib() -> ctypes.CDLL:
         "kv_cache_storage_bytes": (c_sz, [c_int] * 7 + [c_int]),
         "kv_cache_init": (c_int, [ctypes.POINTER(c_p), c_int, c_int, c_int, c_int, c_int, c_int,
                                   ctypes.POINTER(kvcr_rope), c_int, c_p, c_sz]),
+        "kv_cache_storage_bytes_aux": (c_sz, [c_int] * 8 + [c_int]),
+        "kv_cache_init_aux": (c_int, [ctypes.POINTER(c_p), c_int, c_int, c_int, c_int, c_int, c_int,
+                                      c_int, ctypes.POINTER(kvcr_rope), c_int, c_p, c_sz]),
+        "kv_cache_set_aux": (c_int, [c_p, c_p, c_p, i32p, c_int, c_p]),
+        "kv_cache_num_aux": (c_int, [c_p, ctypes.POINTER(c_int)]),
         "kv_cache_append_rope": (c_int, [c_p, c_p, c_p, i32p, c_int, c_p]),
         "kv_cache_evict": (c_int, [c_p, c_int, i32p, c_int, ctypes.POINTER(c_int)]),
         "kv_cache_slot_map": (c_int, [c_p, i32p, c_int]),
@@ -147,6 +155,42 @@ def kv_cache_storage_bytes(sinks, window, tokens_per_frame, heads, head_dim, chu
     return int(lib().kv_cache_storage_bytes(sinks, window, tokens_per_frame, heads, head_dim,
                                             chunk_frames, int(bool(with_rope)),
                                             _dtype_code(dtype)))
+
+
+def kv_cache_storage_bytes_aux(sinks, window, aux_frames, tokens_per_frame, heads, head_dim,
+                               chunk_frames, with_rope, dtype) -> int:
+    return int(lib().kv_cache_storage_bytes_aux(sinks, window, aux_frames, tokens_per_frame, heads,
+                                                head_dim, chunk_frames, int(bool(with_rope)),
+                                                _dtype_code(dtype)))
+
+
+def kv_cache_init_aux(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
+                      rope, dtype, storage) -> ctypes.c_void_p:
+    """Create a cache with ``aux_frames`` auxiliary slots over ``storage``."""
+    h = ctypes.c_void_p()
+    rp = None
+    if rope is not None:
+        rp = ctypes.byref(kvcr_rope(rope.grid_h, rope.grid_w, rope.pairs_t, rope.pairs_h,
+                                    rope.pairs_w, float(rope.base)))
+    ptr = None if storage is None else storage.data_ptr()
+    nbytes = 0 if storage is None else storage.numel() * storage.element_size()
+    _check(lib().kv_cache_init_aux(ctypes.byref(h), sinks, window, aux_frames, tokens_per_frame,
+                                   heads, head_dim, chunk_frames, rp, _dtype_code(dtype), ptr,
+                                   nbytes))
+    return h
+
+
+def kv_cache_set_aux(handle, k, v, aux_pos: Optional[Sequence[int]], n_frames: int,
+                     stream=None) -> None:
+    s = None if (k is None and v is None) else _stream(stream)
+    pos = None if aux_pos is None else _i32(aux_pos)
+    _check(lib().kv_cache_set_aux(handle, _ptr(k), _ptr(v), pos, n_frames, s))
+
+
+def kv_cache_num_aux(handle) -> int:
+    n = ctypes.c_int()
+    _check(lib().kv_cache_num_aux(handle, ctypes.byref(n)))
+    return n.value
 
 
 def kv_cache_init(sinks, window, tokens_per_frame, heads, head_dim, chunk_frames, rope, dtype,
@@ -302,21 +346,23 @@ class Cache:
 
     def __init__(self, sinks: int, window: int, tokens_per_frame: int, heads: int, head_dim: int,
                  chunk_frames: int, rope=None, dtype="bf16", device="cuda",
-                 bookkeeping_only: bool = False):
-        self.sinks, self.window = sinks, window
+                 bookkeeping_only: bool = False, aux_frames: int = 0):
+        self.sinks, self.window, self.aux_frames = sinks, window, aux_frames
         self.T, self.H, self.D, self.F = tokens_per_frame, heads, head_dim, chunk_frames
         self.rope = rope
         self.dtype_code = _dtype_code(dtype)
         self.storage = None
         if not bookkeeping_only:
             import torch
-            nbytes = kv_cache_storage_bytes(sinks, window, tokens_per_frame, heads, head_dim,
-                                            chunk_frames, rope is not None, self.dtype_code)
+            nbytes = kv_cache_storage_bytes_aux(sinks, window, aux_frames, tokens_per_frame, heads,
+                                                head_dim, chunk_frames, rope is not None,
+                                                self.dtype_code)
             if nbytes == 0:
                 raise KvcrError(KVCR_ESHAPE, "invalid cache sizes")
             self.storage = torch.empty(nbytes, dtype=torch.uint8, device=device)
-        self.handle = kv_cache_init(sinks, window, tokens_per_frame, heads, head_dim,
-                                    chunk_frames, rope, self.dtype_code, self.storage)
+        self.handle = kv_cache_init_aux(sinks, window, aux_frames, tokens_per_frame, heads,
+                                        head_dim, chunk_frames, rope, self.dtype_code,
+                                        self.storage)
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -335,6 +381,15 @@ class Cache:
 
     def evict(self, keep_recent: int) -> List[int]:
         return kv_cache_evict(self.handle, keep_recent)
+
+    def set_aux(self, k, v, positions: Optional[Sequence[int]] = None, stream=None) -> None:
+        """Auxiliary frames for the current chunk (dropped by the next append); k, v
+        [n * T, H, D] (None, None on a bookkeeping-only cache with n = len(positions))."""
+        n = (k.shape[0] // self.T) if k is not None else (0 if positions is None else len(positions))
+        kv_cache_set_aux(self.handle, k, v, positions, n, stream)
+
+    def num_aux(self) -> int:
+        return kv_cache_num_aux(self.handle)
 
     def slot_map(self) -> List[int]:
         return kv_cache_slot_map(self.handle, self.sinks + self.window)

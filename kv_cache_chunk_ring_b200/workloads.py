@@ -202,6 +202,19 @@ def rollout_chunks(spec: RolloutSpec, layer: int = 0) -> Iterator[dict]:
             yield dict(chunk=c, step=s, frames=spec.frames_of_chunk(c), q=q, k=k, v=v)
 
 
+def aux_frames(spec: RolloutSpec, chunk: int, n: int, seed_offset: int = 2000):
+    """Auxiliary evidence frames for one chunk: K, V ([n * T, H, D]) and n ascending
+    temporal positions drawn from the frames before the chunk (retrieved history,
+    source-video observations), from PCG64(seed + seed_offset + chunk)."""
+    rng = np.random.Generator(np.random.PCG64(spec.seed + seed_offset + chunk))
+    shape = (n * spec.tokens_per_frame, spec.heads, spec.head_dim)
+    k = draw(rng, shape, spec.dtype)
+    v = draw(rng, shape, spec.dtype)
+    first = spec.frames_of_chunk(chunk)[0]
+    pos = sorted(int(x) for x in rng.integers(0, max(first, 1), size=n))
+    return k, v, pos
+
+
 def text_kv(spec: RolloutSpec) -> Iterator[dict]:
     """Cross-attention inputs: the shared env prompt K/V (drawn once) and, per
     chunk, the chunk's local-prompt K/V and the chunk's cross-attention queries.

@@ -19,9 +19,17 @@ absolute frame index; V is not rotated; the finalized K/V are the last
 step's; with a dynamic window the eviction to W_t happens before the
 chunk's attention and appends use the largest window as capacity.
 
+Auxiliary frames ([WiW] second paragraph: temporary auxiliary attention
+blocks carry extra evidence for the current chunk and are removed once it is
+finalized): ``aux_for(chunk)`` may give K, V of extra frames (and temporal
+positions, at which K is rotated like a cached frame; without positions K is
+used as given); every attention call of that chunk reads them besides the
+cached frames and the chunk itself, and they are never cached.
+
 Parity: pinned (equals brute-force attention over the whole concatenated
 rollout under the set-based visibility rule; a chunk's output does not change
-when later chunks change).
+when later chunks change; auxiliary copies of every visible frame leave O
+unchanged and add ln 2 to LSE; auxiliary frames change only their own chunk).
 """
 from __future__ import annotations
 
@@ -49,12 +57,14 @@ class RolloutResult:
 
 
 def rollout(spec, chunks, rows_for=None, use_rope: bool = True,
-            window_schedule: Optional[List[int]] = None) -> RolloutResult:
+            window_schedule: Optional[List[int]] = None, aux_for=None) -> RolloutResult:
     """Run the rollout of ``spec`` (a RolloutSpec) over ``chunks``.
 
     ``chunks`` yields dicts with chunk, step, frames, q, k, v as produced by
     ``workloads.rollout_chunks``.  ``rows_for(chunk, step)`` returns the query
-    rows to evaluate (default: all).
+    rows to evaluate (default: all).  ``aux_for(chunk)`` returns None or
+    (k_aux, v_aux, positions) with k_aux, v_aux [n * T, H, D] and positions a
+    list of n temporal positions or None.
     """
     T = spec.grid_h * spec.grid_w
     scale = 1.0 / math.sqrt(spec.head_dim)
@@ -80,8 +90,17 @@ def rollout(spec, chunks, rows_for=None, use_rope: bool = True,
         else:
             q_rot, k_rot = q, k
         vis = cache.cached_frames()
-        k_all = np.concatenate([store[f][0] for f in vis] + [k_rot], axis=0)
-        v_all = np.concatenate([store[f][1] for f in vis] + [v], axis=0)
+        k_aux, v_aux = [], []
+        aux = aux_for(c) if aux_for is not None else None
+        if aux is not None and np.asarray(aux[0]).shape[0] > 0:
+            ka = np.asarray(aux[0], dtype=np.float64)
+            va = np.asarray(aux[1], dtype=np.float64)
+            if aux[2] is not None and use_rope:
+                ta, ha, wa = rope_positions(list(aux[2]), spec.grid_h, spec.grid_w)
+                ka = rope3d(ka, ta, ha, wa, pairs, spec.rope().base)
+            k_aux, v_aux = [ka], [va]
+        k_all = np.concatenate([store[f][0] for f in vis] + k_aux + [k_rot], axis=0)
+        v_all = np.concatenate([store[f][1] for f in vis] + v_aux + [v], axis=0)
         rows = np.arange(q.shape[0]) if rows_for is None else np.asarray(rows_for(c, s))
         o, lse = attention(q_rot[rows], k_all, v_all, scale)
         res.outputs.append(o)

@@ -49,20 +49,28 @@ def rope_of(spec):
 
 
 def gpu_rollout(spec, chunks, rows_for: Optional[Callable] = None, use_rope: bool = True,
-                window_schedule: Optional[List[int]] = None):
+                window_schedule: Optional[List[int]] = None, aux_for: Optional[Callable] = None,
+                aux_frames: int = 0):
     """Run the rollout through the C ABI.  Returns dict of per-call outputs (rows
     selected by rows_for, numpy fp64), LSEs, slot maps after each append, and the
-    Cache (for read-back)."""
+    Cache (for read-back).  ``aux_for(chunk)`` -> None or (k, v, positions) sets the
+    chunk's auxiliary frames before its first step (cache built with
+    ``aux_frames`` auxiliary slots)."""
     import torch
     from kv_cache_chunk_ring_b200.kvcr import Cache
     cap = spec.window if window_schedule is None else max(spec.window, max(window_schedule))
     cache = Cache(spec.sinks, cap, spec.tokens_per_frame, spec.heads, spec.head_dim,
-                  spec.chunk_frames, rope=spec.rope() if use_rope else None, dtype=spec.dtype)
+                  spec.chunk_frames, rope=spec.rope() if use_rope else None, dtype=spec.dtype,
+                  aux_frames=aux_frames)
     out = dict(outputs=[], lses=[], slot_maps=[], appended=[], cache=cache)
     for item in chunks:
         c, s, frames = item["chunk"], item["step"], item["frames"]
         if s == 0 and window_schedule is not None:
             cache.evict(window_schedule[c])
+        if s == 0 and aux_for is not None:
+            aux = aux_for(c)
+            if aux is not None:
+                cache.set_aux(to_dev(aux[0], spec.dtype), to_dev(aux[1], spec.dtype), aux[2])
         q = to_dev(item["q"], spec.dtype)
         k = to_dev(item["k"], spec.dtype)
         v = to_dev(item["v"], spec.dtype)

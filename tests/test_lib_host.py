@@ -183,3 +183,41 @@ def test_moba_bwd_rejects_bad_arguments_before_launch():
     bad = kvcr.kvcr_moba_layout(0, 200, 1)
     assert L.moba_attention_bwd(p, p, p, p, p, p, ctypes.byref(bad), 2, 128, kvcr.KVCR_BF16, 0.0,
                                 p, p, p, p, 1 << 30, None) == kvcr.KVCR_ESHAPE
+
+
+def test_aux_slots_bookkeeping():
+    """Auxiliary frames are visible until the chunk's append drops them; they never
+    touch the anchor / window slot table."""
+    c = kvcr.Cache(2, 2, 16, 1, 64, 2, dtype="f32", bookkeeping_only=True, aux_frames=3)
+    ref = kvcr.Cache(2, 2, 16, 1, 64, 2, dtype="f32", bookkeeping_only=True)
+    assert c.num_aux() == 0
+    for ch in range(5):
+        frames = [2 * ch, 2 * ch + 1]
+        n = ch % 4
+        if n <= 3:
+            c.set_aux(None, None, positions=list(range(n)))
+            assert c.num_aux() == n
+        c.append(None, None, frames)
+        ref.append(None, None, frames)
+        assert c.num_aux() == 0
+        assert c.slot_map() == ref.slot_map()
+    with pytest.raises(kvcr.KvcrError) as e:
+        c.set_aux(None, None, positions=[0, 1, 2, 3])        # more than aux_frames
+    assert e.value.code == kvcr.KVCR_ESHAPE
+    assert c.num_aux() == 0
+    with pytest.raises(kvcr.KvcrError) as e:
+        c.set_aux(None, None, positions=[0, -1])
+    assert e.value.code == kvcr.KVCR_EINVAL
+    c.set_aux(None, None, positions=[4, 5])
+    c.set_aux(None, None, positions=[])                        # n = 0 drops them now
+    assert c.num_aux() == 0
+
+
+def test_aux_storage_bytes():
+    T, H, D, F = 1508, 12, 128, 4
+    base = kvcr.kv_cache_storage_bytes(6, 8, T, H, D, F, True, "bf16")
+    assert kvcr.kv_cache_storage_bytes_aux(6, 8, 0, T, H, D, F, True, "bf16") == base
+    frame = T * H * D * 2
+    grown = kvcr.kv_cache_storage_bytes_aux(6, 8, 4, T, H, D, F, True, "bf16")
+    assert base + 2 * 4 * frame <= grown <= base + 2 * 4 * frame + 2 * 256
+    assert kvcr.kv_cache_storage_bytes_aux(6, 8, 19, T, H, D, F, True, "bf16") == 0  # > 32 slots
