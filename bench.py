@@ -502,17 +502,34 @@ def run_layers30(args) -> dict:
             c.append(k, v, frames)
         frame[0] += F
 
+    def chunk_batched():
+        # the same chunk with the 30 appends done by one batched launch at its end
+        frames = list(range(frame[0], frame[0] + F))
+        ks, vs = [], []
+        for li, c in enumerate(caches):
+            for s in range(spec.steps):
+                q, k, v = pool[n_call[0] % len(pool)]
+                n_call[0] += 1
+                c.attention(q, k, v, frames, out=o)
+            ks.append(k)
+            vs.append(v)
+        kvcr.append_batch(caches, ks, vs, frames)
+        frame[0] += F
+
     for _ in range(STEADY_CHUNK):
         chunk()
     kvcr.kvcr_trace_reset()
     ms = _timed(chunk, args.steps, args.warmup)
+    ms_batched = _timed(chunk_batched, args.steps, args.warmup)
     kvcr.kvcr_trace_enable(True)
     chunk()
+    chunk_batched()
     torch.cuda.synchronize()
     kvcr.kvcr_trace_enable(False)
     kt = {name: kvcr.kvcr_trace_read(kid) for kid, name in kvcr.KERNEL_NAMES.items()}
     kvcr.kvcr_trace_reset()
     flops = spec.layers * spec.steps * step_flops(spec)
+    bat_n, bat_ms = kt["append_batch"]
     app_n, app_ms = kt["append_rope"]
     return {"workload": spec.name, "ms_per_chunk": round(ms, 3),
             "attention_tflops_per_chunk": round(flops / 1e12, 2),
@@ -520,6 +537,10 @@ def run_layers30(args) -> dict:
             "attn_kernel_ms": round(kt["chunk_attn"][1] / max(1, kt["chunk_attn"][0]), 4),
             "append_kernel_us": round(1e3 * app_ms / max(1, app_n), 2),
             "append_gb_s": round(append_bytes(spec) / (app_ms / max(1, app_n) * 1e-3) / 1e9, 1),
+            "ms_per_chunk_batched_append": round(ms_batched, 3),
+            "append_batch_kernel_us": round(1e3 * bat_ms / max(1, bat_n), 2),
+            "append_batch_gb_s": round(spec.layers * append_bytes(spec) /
+                                       (bat_ms / max(1, bat_n) * 1e-3) / 1e9, 1),
             "steps": args.steps, "warmup": args.warmup,
             "note": "steady-state chunks (cache full); 30 independent layer caches, 5.0 GB"}
 

@@ -160,6 +160,20 @@ int kv_cache_num_aux(const kvcr_cache *c, int *n);
 int kv_cache_append_rope(kvcr_cache *c, const void *k, const void *v,
                          const int32_t *frame_idx, int n_frames, void *stream);
 
+/* kv_cache_append_rope() of the same frames into several caches (e.g. every
+ * layer's cache at the end of a chunk) in one launch.  caches: host array of
+ * n_caches distinct handles with the same tokens_per_frame, heads, head_dim,
+ * dtype and RoPE (and all with storage, or all bookkeeping-only); k[i], v[i]:
+ * device [n_frames * tokens_per_frame][heads][head_dim] for cache i (host
+ * arrays of device pointers; NULL arrays for bookkeeping-only caches).  Each
+ * cache's slot table, written K / V and last-append record end up exactly as
+ * after kv_cache_append_rope() on it alone.  n_caches * n_frames <= 256.  Errors
+ * (checked for every cache before anything changes): KVCR_EINVAL, KVCR_ESHAPE
+ * (mismatched caches, sizes), KVCR_ESTATE (frame order). */
+int kv_cache_append_rope_batch(kvcr_cache *const *caches, int n_caches, const void *const *k,
+                               const void *const *v, const int32_t *frame_idx, int n_frames,
+                               void *stream);
+
 /* Dynamic window: evict the oldest non-anchor frames until at most keep_recent
  * remain (0 <= keep_recent <= window).  Host only.  evicted_out (nullable) receives
  * up to evicted_cap evicted frame indices, oldest first; *n_evicted (nullable)
@@ -302,7 +316,8 @@ enum {
     KVCR_K_MOBA_BWD_DKDV = 6, /* MoBA backward: dK and dV (tensor cores) */
     KVCR_K_MOBA_BWD_DQ = 7,   /* MoBA backward: dQ (tensor cores) */
     KVCR_K_SET_AUX = 8,       /* auxiliary frames written into their slots (RoPE3D of K) */
-    KVCR_K_COUNT = 9
+    KVCR_K_APPEND_BATCH = 9,  /* one cache write for several caches (RoPE3D of K) */
+    KVCR_K_COUNT = 10
 };
 
 /* Count of every kernel the library launched in this process. */

@@ -31,6 +31,7 @@
 #include "attn_bwd.h"
 #include "kvcr_internal.h"
 #include "moba_layout.h"
+#include "rope_batch.h"
 #include "static_scratch.h"
 
 using namespace kvcr;
@@ -503,6 +504,110 @@ int kv_cache_append_rope(kvcr_cache* c, const void* k, const void* v, const int3
   c->last_slots = slots;
   c->last_evicted = evicted;
   c->n_aux = 0;  // the chunk is finalized: its auxiliary frames are dropped
+  return KVCR_OK;
+}
+
+int kv_cache_append_rope_batch(kvcr_cache* const* caches, int n_caches, const void* const* k,
+                               const void* const* v, const int32_t* frame_idx, int n_frames,
+                               void* stream) {
+  const char* fn = "kv_cache_append_rope_batch";
+  if (caches == nullptr || n_caches < 1) return fail(KVCR_EINVAL, std::string(fn) + ": no caches");
+  if (n_frames < 0 || n_frames > kMaxFrames)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_frames must be in [0, 16]");
+  if ((long long)n_caches * n_frames > kMaxBatchPairs)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_caches * n_frames must be <= 256");
+  const kvcr_cache* c0 = caches[0];
+  for (int i = 0; i < n_caches; ++i) {
+    const kvcr_cache* c = caches[i];
+    if (c == nullptr) return fail(KVCR_EINVAL, std::string(fn) + ": a cache is NULL");
+    for (int j = 0; j < i; ++j)
+      if (caches[j] == c) return fail(KVCR_EINVAL, std::string(fn) + ": a cache is listed twice");
+    if (c->T != c0->T || c->H != c0->H || c->D != c0->D || c->dtype != c0->dtype ||
+        c->rope != c0->rope || c->has_storage != c0->has_storage ||
+        (c->rope && (c->rp.grid_h != c0->rp.grid_h || c->rp.grid_w != c0->rp.grid_w ||
+                     c->rp.pairs_t != c0->rp.pairs_t || c->rp.pairs_h != c0->rp.pairs_h ||
+                     c->rp.pairs_w != c0->rp.pairs_w || c->rp.base != c0->rp.base)))
+      return fail(KVCR_ESHAPE, std::string(fn) +
+                                   ": caches differ in frame shape, dtype, RoPE or storage");
+    int rc = check_frames(c, frame_idx, n_frames, fn);
+    if (rc) return rc;
+    if (c->has_storage && n_frames > 0) {
+      if (k == nullptr || v == nullptr || k[i] == nullptr || v[i] == nullptr)
+        return fail(KVCR_EINVAL, std::string(fn) + ": k/v NULL");
+      if (!aligned16(k[i]) || !aligned16(v[i]))
+        return fail(KVCR_EINVAL, std::string(fn) + ": k/v must be 16-byte aligned");
+    } else if (!c->has_storage && k != nullptr && v != nullptr && (k[i] != nullptr || v[i] != nullptr)) {
+      return fail(KVCR_ESTATE, std::string(fn) + ": bookkeeping-only caches take k = v = NULL");
+    }
+  }
+  if (n_frames == 0) {
+    for (int i = 0; i < n_caches; ++i) {
+      caches[i]->last_slots.clear();
+      caches[i]->last_evicted.clear();
+      caches[i]->n_aux = 0;
+    }
+    return KVCR_OK;
+  }
+  std::vector<SlotState> before;
+  std::vector<std::vector<int>> slots(n_caches), evicted(n_caches);
+  for (int i = 0; i < n_caches; ++i) {
+    before.push_back(snapshot(caches[i]));
+    slots[i].resize(n_frames);
+    for (int f = 0; f < n_frames; ++f) slots[i][f] = place_frame(caches[i], frame_idx[f], evicted[i]);
+  }
+  if (c0->has_storage) {
+    RopeCopyBatchParams* p = new RopeCopyBatchParams();
+    std::memset(p, 0, sizeof(*p));
+    p->T = c0->T;
+    p->H = c0->H;
+    p->D = c0->D;
+    p->grid_w = c0->rope ? c0->rp.grid_w : 1;
+    p->rotate_a = c0->rope ? 1 : 0;
+    p->pairs_t = c0->rope ? c0->rp.pairs_t : 0;
+    p->pairs_h = c0->rope ? c0->rp.pairs_h : 0;
+    p->pairs_w = c0->rope ? c0->rp.pairs_w : 0;
+    p->htab = c0->rope ? reinterpret_cast<const float2*>(c0->storage + c0->lay.h_off) : nullptr;
+    p->wtab = c0->rope ? reinterpret_cast<const float2*>(c0->storage + c0->lay.w_off) : nullptr;
+    if (c0->rope)
+      for (int f = 0; f < n_frames; ++f)
+        for (int j = 0; j < c0->rp.pairs_t; ++j) {
+          const double ang = (double)frame_idx[f] *
+                             std::pow(c0->rp.base, -(2.0 * j) / (2.0 * c0->rp.pairs_t));
+          p->ttab[f][j] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+        }
+    const size_t frame_bytes = (size_t)c0->T * c0->H * c0->D * c0->esize;
+    int n = 0;
+    for (int i = 0; i < n_caches; ++i) {
+      const kvcr_cache* c = caches[i];
+      for (int f = 0; f < n_frames; ++f) {
+        // skip frames not retained, or evicted again by a later frame of this call
+        if (slots[i][f] < 0 || c->slot_frame[slots[i][f]] != frame_idx[f]) continue;
+        p->src_a[n] = static_cast<const uint8_t*>(k[i]) + (size_t)f * frame_bytes;
+        p->src_b[n] = static_cast<const uint8_t*>(v[i]) + (size_t)f * frame_bytes;
+        p->dst_a[n] = c->storage + c->lay.k_off + (size_t)slots[i][f] * frame_bytes;
+        p->dst_b[n] = c->storage + c->lay.v_off + (size_t)slots[i][f] * frame_bytes;
+        p->tframe[n] = f;
+        ++n;
+      }
+    }
+    p->n = n;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    {
+      LaunchScope scope(KVCR_K_APPEND_BATCH, s);
+      e = launch_rope_copy_batch(*p, c0->dtype, s, c0->n_sm);
+    }
+    delete p;
+    if (e != cudaSuccess) {
+      for (int i = 0; i < n_caches; ++i) restore(caches[i], before[i]);
+      return cuda_fail(e, "kv_cache_append_rope_batch: launch");
+    }
+  }
+  for (int i = 0; i < n_caches; ++i) {
+    caches[i]->last_slots = slots[i];
+    caches[i]->last_evicted = evicted[i];
+    caches[i]->n_aux = 0;
+  }
   return KVCR_OK;
 }
 

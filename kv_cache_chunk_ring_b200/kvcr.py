@@ -23,17 +23,18 @@ KVCR_BF16, KVCR_F32 = 0, 1
 KVCR_TILE_EMPTY, KVCR_TILE_PARTIAL, KVCR_TILE_FULL = 0, 1, 2
 (KVCR_K_APPEND_ROPE, KVCR_K_ROPE_STAGE, KVCR_K_CHUNK_ATTN, KVCR_K_MOBA_ATTN,
  KVCR_K_ATTN_F32, KVCR_K_MOBA_BWD_PREP, KVCR_K_MOBA_BWD_DKDV, KVCR_K_MOBA_BWD_DQ,
- KVCR_K_SET_AUX) = range(9)
+ KVCR_K_SET_AUX, KVCR_K_APPEND_BATCH) = range(10)
 KERNEL_NAMES = {KVCR_K_APPEND_ROPE: "append_rope", KVCR_K_ROPE_STAGE: "rope_stage",
                 KVCR_K_CHUNK_ATTN: "chunk_attn", KVCR_K_MOBA_ATTN: "moba_attn",
                 KVCR_K_ATTN_F32: "attn_f32", KVCR_K_MOBA_BWD_PREP: "moba_bwd_prep",
                 KVCR_K_MOBA_BWD_DKDV: "moba_bwd_dkdv", KVCR_K_MOBA_BWD_DQ: "moba_bwd_dq",
-                KVCR_K_SET_AUX: "set_aux"}
+                KVCR_K_SET_AUX: "set_aux", KVCR_K_APPEND_BATCH: "append_batch"}
 
 # every symbol include/kvcr.h declares
 EXPORTS = [
     "kv_cache_storage_bytes", "kv_cache_init", "kv_cache_storage_bytes_aux", "kv_cache_init_aux",
-    "kv_cache_set_aux", "kv_cache_num_aux", "kv_cache_append_rope", "kv_cache_evict",
+    "kv_cache_set_aux", "kv_cache_num_aux", "kv_cache_append_rope", "kv_cache_append_rope_batch",
+    "kv_cache_evict",
     "kv_cache_slot_map", "kv_cache_last_append", "kv_cache_num_cached", "kv_cache_slot_data",
     "kv_cache_destroy",
     "chunk_attention_fwd", "chunk_attention_fwd_static_scratch", "moba_attention_fwd",
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
         "kv_cache_set_aux": (c_int, [c_p, c_p, c_p, i32p, c_int, c_p]),
         "kv_cache_num_aux": (c_int, [c_p, ctypes.POINTER(c_int)]),
         "kv_cache_append_rope": (c_int, [c_p, c_p, c_p, i32p, c_int, c_p]),
+        "kv_cache_append_rope_batch": (c_int, [ctypes.POINTER(c_p), c_int, ctypes.POINTER(c_p),
+                                               ctypes.POINTER(c_p), i32p, c_int, c_p]),
         "kv_cache_evict": (c_int, [c_p, c_int, i32p, c_int, ctypes.POINTER(c_int)]),
         "kv_cache_slot_map": (c_int, [c_p, i32p, c_int]),
         "kv_cache_last_append": (c_int, [c_p, i32p, c_int, i32p, c_int, ctypes.POINTER(c_int)]),
@@ -212,6 +215,26 @@ def kv_cache_append_rope(handle, k, v, frame_idx: Sequence[int], stream=None) ->
     n = len(frame_idx)
     s = None if (k is None and v is None) else _stream(stream)
     _check(lib().kv_cache_append_rope(handle, _ptr(k), _ptr(v), _i32(frame_idx), n, s))
+
+
+def kv_cache_append_rope_batch(handles, ks, vs, frame_idx: Sequence[int], stream=None) -> None:
+    """One launch appending the same frames to several caches (ks[i], vs[i] for handles[i];
+    ks = vs = None for bookkeeping-only caches)."""
+    n = len(handles)
+    hs = (ctypes.c_void_p * n)(*[h.value if isinstance(h, ctypes.c_void_p) else h for h in handles])
+    if ks is None:
+        kp = vp = None
+        s = None
+    else:
+        kp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in ks])
+        vp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in vs])
+        s = _stream(stream)
+    _check(lib().kv_cache_append_rope_batch(hs, n, kp, vp, _i32(frame_idx), len(frame_idx), s))
+
+
+def append_batch(caches, ks, vs, frames: Sequence[int], stream=None) -> None:
+    """Cache-level wrapper of kv_cache_append_rope_batch."""
+    kv_cache_append_rope_batch([c.handle for c in caches], ks, vs, frames, stream)
 
 
 def kv_cache_evict(handle, keep_recent: int) -> List[int]:

@@ -221,3 +221,38 @@ def test_aux_storage_bytes():
     grown = kvcr.kv_cache_storage_bytes_aux(6, 8, 4, T, H, D, F, True, "bf16")
     assert base + 2 * 4 * frame <= grown <= base + 2 * 4 * frame + 2 * 256
     assert kvcr.kv_cache_storage_bytes_aux(6, 8, 19, T, H, D, F, True, "bf16") == 0  # > 32 slots
+
+
+def test_batched_append_bookkeeping_matches_single_appends():
+    caches = [kvcr.Cache(2, 3, 16, 1, 64, 2, dtype="f32", bookkeeping_only=True) for _ in range(3)]
+    twins = [kvcr.Cache(2, 3, 16, 1, 64, 2, dtype="f32", bookkeeping_only=True) for _ in range(3)]
+    caches[1].append(None, None, [0])
+    twins[1].append(None, None, [0])
+    for ch in range(1, 7):
+        frames = [2 * ch, 2 * ch + 1]
+        if ch == 4:
+            caches[2].evict(1)
+            twins[2].evict(1)
+        kvcr.append_batch(caches, None, None, frames)
+        for c, t in zip(caches, twins):
+            t.append(None, None, frames)
+            assert c.slot_map() == t.slot_map()
+            assert kvcr.kv_cache_last_append(c.handle, 2) == kvcr.kv_cache_last_append(t.handle, 2)
+
+
+def test_batched_append_rejects_before_changing_anything():
+    a = kvcr.Cache(2, 2, 16, 1, 64, 2, dtype="f32", bookkeeping_only=True)
+    b = kvcr.Cache(2, 2, 16, 1, 64, 2, dtype="f32", bookkeeping_only=True)
+    other = kvcr.Cache(2, 2, 25, 1, 64, 2, dtype="f32", bookkeeping_only=True)
+    b.append(None, None, [0, 1, 2])
+    before = (a.slot_map(), b.slot_map())
+    with pytest.raises(kvcr.KvcrError) as e:          # b already holds frame 2
+        kvcr.append_batch([a, b], None, None, [1, 2])
+    assert e.value.code == kvcr.KVCR_ESTATE
+    with pytest.raises(kvcr.KvcrError) as e:
+        kvcr.append_batch([a, other], None, None, [5])
+    assert e.value.code == kvcr.KVCR_ESHAPE
+    with pytest.raises(kvcr.KvcrError) as e:
+        kvcr.append_batch([a, a], None, None, [5])
+    assert e.value.code == kvcr.KVCR_EINVAL
+    assert (a.slot_map(), b.slot_map()) == before
