@@ -50,6 +50,8 @@ __device__ int g_bwd_status = 0;
 namespace {
 using namespace ptx;
 
+constexpr int kMaxDevices = 64;
+
 constexpr int kStages = 2;
 constexpr int kThreads = 384;
 // launch 384 x 168 registers; producer warpgroup 80, the two work warpgroups
@@ -748,12 +750,16 @@ __global__ void __launch_bounds__(256) moba_bwd_prep_kernel(const MobaBwdPrepPar
 template <int HD>
 cudaError_t launch_dkdv(const MobaBwdParams& p, cudaStream_t s) {
   auto kern = moba_dkdv_kernel<HD>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the shared-memory limit is a per-device attribute of the function
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<HD>::kBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev] = true;
   }
   kern<<<(unsigned)(p.s.n_units * p.H), kThreads, BwdSmem<HD>::kBytes, s>>>(p);
   return cudaGetLastError();
@@ -762,12 +768,16 @@ cudaError_t launch_dkdv(const MobaBwdParams& p, cudaStream_t s) {
 template <int HD>
 cudaError_t launch_dq(const MobaBwdParams& p, cudaStream_t s) {
   auto kern = moba_dq_kernel<HD>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the shared-memory limit is a per-device attribute of the function
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<HD>::kBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev] = true;
   }
   kern<<<(unsigned)(p.s.n_units * p.H), kThreads, BwdSmem<HD>::kBytes, s>>>(p);
   return cudaGetLastError();

@@ -51,6 +51,8 @@ __device__ int g_attn_status = 0;
 namespace {
 using namespace ptx;
 
+constexpr int kMaxDevices = 64;
+
 constexpr int kStages = 2;
 constexpr int kThreads = 384;
 // Register budgets after setmaxnreg: launch 384 x 168; producer warpgroup
@@ -641,12 +643,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 template <int HD, bool kMoba, typename Params>
 cudaError_t launch_impl(const Params& p, dim3 grid, cudaStream_t s) {
   auto kern = attn_fwd_kernel<HD, kMoba, Params>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the shared-memory limit is a per-device attribute of the function
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<HD>::kBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev] = true;
   }
   kern<<<grid, kThreads, Smem<HD>::kBytes, s>>>(p);
   return cudaGetLastError();
