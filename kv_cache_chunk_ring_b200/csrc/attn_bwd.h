@@ -6,7 +6,8 @@
 namespace kvcr {
 
 // Work order of one backward launch: 128-row tiles (key tiles for dK / dV,
-// query tiles for dQ), heaviest first.  CTA b runs tile order[b / H] of head b % H.
+// query tiles for dQ), heaviest first.  CTA b runs tile order[b % n_units] of
+// head b / n_units (head-major, so co-resident CTAs share one head's tiles in L2).
 struct MobaBwdSched {
   int n_chunks, chunk_tokens, n_bidir;
   int L;

@@ -14,7 +14,8 @@
 //   prep   per head and 128-row tile: LSE_i * log2 e of its rows, then D_i of
 //          them (ws[h][t][0][r], ws[h][t][1][r]); rows past L get (+inf, 0), so
 //          their probabilities are exactly 0.
-//   dK/dV  one CTA per (head, 128-key tile); K_j, V_j stay in shared memory and
+//   dK/dV  one CTA per (head, 128-key tile), head-major and heaviest tiles first
+//          within a head; K_j, V_j stay in shared memory and
 //          the query tiles that may read them stream through a 2-stage ring:
 //            S^T  = K_j Q_i^T            (SS)       TMEM cols   0-127
 //            dP^T = V_j dO_i^T           (SS)       TMEM cols 128-255
@@ -316,8 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
   BwdCtl* ctl = reinterpret_cast<BwdCtl*>(smem + L::kCtl);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int kt = p.s.order[blockIdx.x / p.H];
-  const int h = blockIdx.x % p.H;
+  const int h = blockIdx.x / p.s.n_units;             // head-major: co-resident CTAs
+  const int kt = p.s.order[blockIdx.x - h * p.s.n_units];  // share one head in L2
   const int k0 = kt * kTile;
 
   bwd_setup<true>(p, ctl, kt, warp, lane);
@@ -523,8 +524,8 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
   BwdCtl* ctl = reinterpret_cast<BwdCtl*>(smem + L::kCtl);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = p.s.order[blockIdx.x / p.H];
-  const int h = blockIdx.x % p.H;
+  const int h = blockIdx.x / p.s.n_units;             // head-major: co-resident CTAs
+  const int qt = p.s.order[blockIdx.x - h * p.s.n_units];  // share one head in L2
   const int q0 = qt * kTile;
 
   bwd_setup<false>(p, ctl, qt, warp, lane);
