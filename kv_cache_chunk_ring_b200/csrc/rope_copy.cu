@@ -149,17 +149,78 @@ __device__ __forceinline__ void copy_frame(const Elem* src_a, const Elem* src_b,
   }
 }
 
+// The single-cache kernel keeps its own copy of the loop: reading the frame's
+// parameters straight from the kernel parameters measured ~5 % faster than
+// passing them to copy_frame().
 template <typename Elem, int D>
 __global__ void __launch_bounds__(256) rope_copy_kernel(const __grid_constant__ RopeCopyParams p) {
+  constexpr int kPerVec = 16 / sizeof(Elem);          // elements per 16-byte vector
+  constexpr int kPairsPerVec = kPerVec / 2;
+  constexpr int kVecPerRow = D / kPerVec;             // vectors per (token, head)
+  constexpr int kBatch = 6;                           // vectors in flight per lane and tensor
   const int f = blockIdx.y;                           // destination frame
-  const long long frame_elems = (long long)p.T * p.H * D;
-  copy_frame<Elem, D>(static_cast<const Elem*>(p.src_a) + p.src_frame[f] * frame_elems,
-                      static_cast<const Elem*>(p.src_b) + p.src_frame[f] * frame_elems,
-                      static_cast<Elem*>(p.dst_a) + p.dst_frame_off[f],
-                      static_cast<Elem*>(p.dst_b) + p.dst_frame_off[f], p.ttab[f], p.T, p.H,
-                      p.grid_w, p.pairs_t, p.pairs_h, p.pairs_w, p.htab, p.wtab, p.rotate_a,
-                      p.rotate_b, blockIdx.x, gridDim.x);
+  const int lane = threadIdx.x & 31;
+  const int vpt = p.H * kVecPerRow;                   // vectors per token
+  const int n_mine = (vpt - lane + 31) / 32;          // vectors of this lane per token
+  const int pair0 = (lane % kVecPerRow) * kPairsPerVec;
+  const long long tok_elems = (long long)p.H * D;
+  const Elem* src_a = static_cast<const Elem*>(p.src_a) + (long long)p.src_frame[f] * p.T * tok_elems;
+  const Elem* src_b = static_cast<const Elem*>(p.src_b) + (long long)p.src_frame[f] * p.T * tok_elems;
+  Elem* dst_a = static_cast<Elem*>(p.dst_a) + p.dst_frame_off[f];
+  Elem* dst_b = static_cast<Elem*>(p.dst_b) + p.dst_frame_off[f];
+
+  // axis and index of this lane's pairs; t-axis (cos, sin) are per frame
+  int axis[4], jx[4];
+  float2 cs_t[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    int i = pair0 + k;
+    axis[k] = i < p.pairs_t ? 0 : (i < p.pairs_t + p.pairs_h ? 1 : 2);
+    jx[k] = axis[k] == 0 ? i : (axis[k] == 1 ? i - p.pairs_t : i - p.pairs_t - p.pairs_h);
+    cs_t[k] = (k < kPairsPerVec && axis[k] == 0 && (p.rotate_a || p.rotate_b))
+                  ? p.ttab[f][jx[k] < kMaxPairsT ? jx[k] : 0]
+                  : make_float2(1.f, 0.f);
+  }
+  const int warps_total = gridDim.x * (blockDim.x / 32);
+  for (int tok = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); tok < p.T;
+       tok += warps_total) {
+    float2 cs[4];
+    if (p.rotate_a || p.rotate_b) {
+      const int hh = tok / p.grid_w;
+      const int ww = tok - hh * p.grid_w;
+#pragma unroll
+      for (int k = 0; k < kPairsPerVec; ++k) {
+        if (axis[k] == 0) cs[k] = cs_t[k];
+        else if (axis[k] == 1) cs[k] = p.htab[hh * p.pairs_h + jx[k]];
+        else cs[k] = p.wtab[ww * p.pairs_w + jx[k]];
+      }
+    }
+    const long long base = (long long)tok * tok_elems;
+    for (int k0 = 0; k0 < n_mine; k0 += kBatch) {
+      uint4 a[kBatch], b[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        if (k0 + k < n_mine) {
+          const long long off = base + (long long)(lane + 32 * (k0 + k)) * kPerVec;
+          a[k] = ld_stream(src_a + off);
+          b[k] = ld_stream(src_b + off);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        if (k0 + k < n_mine) {
+          const long long off = base + (long long)(lane + 32 * (k0 + k)) * kPerVec;
+          uint4 ra = a[k], rb = b[k];
+          if (p.rotate_a) ra = rotate_vec<kPairsPerVec>(ra, cs);
+          if (p.rotate_b) rb = rotate_vec<kPairsPerVec>(rb, cs);
+          st_vec(dst_a + off, ra);
+          st_vec(dst_b + off, rb);
+        }
+      }
+    }
+  }
 }
+
 
 // Several caches at once: blockIdx.y = one (cache, frame) pair of the batch.
 template <typename Elem, int D>
