@@ -408,7 +408,14 @@ class Cache:
     def set_aux(self, k, v, positions: Optional[Sequence[int]] = None, stream=None) -> None:
         """Auxiliary frames for the current chunk (dropped by the next append); k, v
         [n * T, H, D] (None, None on a bookkeeping-only cache with n = len(positions))."""
-        n = (k.shape[0] // self.T) if k is not None else (0 if positions is None else len(positions))
+        if k is not None:
+            if k.shape != v.shape or k.shape[0] % self.T or tuple(k.shape[1:]) != (self.H, self.D):
+                raise ValueError(f"aux k, v must both be [n * {self.T}, {self.H}, {self.D}]")
+            n = k.shape[0] // self.T
+            if positions is not None and len(positions) != n:
+                raise ValueError("one position per auxiliary frame")
+        else:
+            n = 0 if positions is None else len(positions)
         kv_cache_set_aux(self.handle, k, v, positions, n, stream)
 
     def num_aux(self) -> int:
