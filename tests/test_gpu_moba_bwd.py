@@ -168,7 +168,9 @@ def test_full_size_sampled():
     sum_do = do.astype(np.float64).sum(0)
     for h in range(H):
         nk = float(dk[:, h].float().norm())
-        nv = float(dv[:, h].float().norm())
+        # P is a bf16 operand: each row's sum is off by up to 2^-9, so sum_j dV_j - sum_i dO_i
+        # is a random walk of size ~2^-9 ||dO||_F (bounded here with a factor 4)
+        bound_v = 4 * 2.0 ** -9 * float(np.linalg.norm(do[:, h]))
         assert np.linalg.norm(sum_dk[h]) <= 1e-2 * nk, (h, np.linalg.norm(sum_dk[h]), nk)
-        assert np.linalg.norm(sum_dv[h] - sum_do[h]) <= 1e-2 * nv, \
-            (h, np.linalg.norm(sum_dv[h] - sum_do[h]), nv)
+        assert np.linalg.norm(sum_dv[h] - sum_do[h]) <= bound_v, \
+            (h, np.linalg.norm(sum_dv[h] - sum_do[h]), bound_v)

@@ -256,3 +256,16 @@ def test_batched_append_rejects_before_changing_anything():
         kvcr.append_batch([a, a], None, None, [5])
     assert e.value.code == kvcr.KVCR_EINVAL
     assert (a.slot_map(), b.slot_map()) == before
+
+
+def test_moba_longest_sequence_accepted_and_one_more_rejected():
+    """The MoBA calls take sequences of up to 4096 tiles of 128 tokens (524288)."""
+    import ctypes
+    assert kvcr.moba_attention_bwd_workspace_bytes(16, 16384, 0, 1) == 4096 * 128 * 8
+    assert kvcr.moba_attention_bwd_workspace_bytes(16, 16384, 0, 1) > 0
+    assert kvcr.moba_attention_bwd_workspace_bytes(16, 16385, 0, 1) == 0
+    with pytest.raises(kvcr.KvcrError) as e:
+        kvcr.moba_classify_tiles(16, 16385, 0, 128)
+    assert e.value.code == kvcr.KVCR_ESHAPE
+    cls = kvcr.moba_classify_tiles(16, 16384, 0, 128)
+    assert cls.shape == (4096, 4096)
