@@ -27,6 +27,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -116,7 +117,7 @@ class ClockSampler:
         ids = [x.strip() for x in vis.split(",") if x.strip()]
         self.dev = ids[device_index] if device_index < len(ids) else str(device_index)
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"kvcr_clocks_{os.getpid()}.csv")
 
     def start(self):
         try:
