@@ -1,4 +1,4 @@
-"""CPU oracle for the sink + window chunk-attention path and the MoBA mask.
+"""CPU oracle for the sink + window chunk-attention path, the MoBA mask and its backward.
 
 TEST INFRASTRUCTURE ONLY.  This package is a plain, slow, fp64 restatement of
 what the method computes.  Only the test suite, the package smoke check and
@@ -24,7 +24,9 @@ Sources (web pages; cited by title and section):
          each chunk".
   [WiW]  "Westlake AGI Lab's 'World in World' Steers Frozen Video Models" --
          second paragraph: 18 latent-frame slots = 6 anchors + 8 recent + 4
-         current; initial observation + recently finalized outputs.
+         current; initial observation + recently finalized outputs; temporary
+         auxiliary attention blocks for the current chunk, removed once it is
+         finalized.
   [RT]   kaarelkaarelson.com/lingbot (LingBot-World 2.0 in real time on one
          RTX 5090) -- setup paragraph (832x464, four denoising steps,
          16-frame chunks) and the step / kernel tables.
@@ -41,3 +43,5 @@ from .moba import (MobaLayout, block_of, moba_allowed, moba_mask, classify_tiles
                    classify_tiles_blocks, moba_attention_rows, TILE_EMPTY, TILE_PARTIAL,
                    TILE_FULL)
 from .rollout import rollout, RolloutResult  # noqa: F401
+from .moba_bwd import (attention_bwd_masked, moba_bwd_dense, moba_dq_rows,  # noqa: F401
+                       moba_dkdv_keys)
