@@ -108,3 +108,20 @@ def test_planted_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(mb, "attention_bwd_masked", no_d)
     with pytest.raises(AssertionError):
         test_matches_central_finite_differences(2, 3, 1)
+
+
+def test_single_readable_key_closed_form():
+    """n = 1, one-token chunks, no bidirectional block: the query of C1 reads only C1's key
+    and the query of N1 only N1's (N1 reads no clean chunk before it).  P = 1 on that key,
+    O = its V, dP = dO . V = D, so dS = 0: dV = dO, dQ = dK = 0."""
+    lay = MobaLayout(1, 1, 0)
+    q, k, v, do = _inputs(lay, H=3, D=5, seed=11)
+    dq, dk, dv = mb.moba_bwd_dense(q, k, v, do, lay, 0.6)
+    np.testing.assert_allclose(dv, do, atol=1e-12)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-12)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-12)
+    rows = [0, 1]
+    np.testing.assert_allclose(mb.moba_dq_rows(q, k, v, do, lay, rows, 0.6), 0.0, atol=1e-12)
+    dk_s, dv_s = mb.moba_dkdv_keys(q, k, v, do, lay, rows, 0.6)
+    np.testing.assert_allclose(dv_s, do, atol=1e-12)
+    np.testing.assert_allclose(dk_s, 0.0, atol=1e-12)
