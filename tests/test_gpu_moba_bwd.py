@@ -63,7 +63,8 @@ def _gpu_fwd_bwd(spec, inputs=None):
 @pytest.mark.parametrize("n,c,m,H,D", [(1, 200, 1, 2, 128), (2, 200, 1, 2, 128),
                                        (3, 100, 2, 2, 64), (2, 128, 1, 1, 128),
                                        (3, 77, 0, 2, 128), (4, 50, 3, 2, 128),
-                                       (1, 5, 0, 1, 128), (2, 300, 2, 1, 64)])
+                                       (1, 5, 0, 1, 128), (2, 300, 2, 1, 64),
+                                       (1, 1, 0, 1, 128), (1, 1, 0, 2, 64)])   # one key per query
 def test_small_layouts_every_gradient(n, c, m, H, D):
     spec = wl.MobaSpec("t", heads=H, head_dim=D, n_chunks=n, chunk_tokens=c, n_bidir_chunks=m,
                        seed=60 + n + c + m)
