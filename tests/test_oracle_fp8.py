@@ -1,0 +1,99 @@
+"""Pins of the oracle's e4m3 quantization and the low-precision QK^T attention."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import fp8
+from oracle.attn import attention
+
+
+def test_code_table_from_the_format():
+    vals = fp8.e4m3_values()
+    assert vals[0] == 0.0 and vals[1] == 2.0 ** -9 and vals[7] == 7 * 2.0 ** -9
+    assert vals[8] == 2.0 ** -6                         # smallest normal: exponent 1
+    assert vals[0x38] == 1.0                            # exponent 7 (bias), mantissa 0
+    assert vals[126] == 448.0 and np.isnan(vals[127]) and np.isnan(vals[255])
+    assert vals[128 + 0x38] == -1.0
+    finite = vals[:127]
+    assert np.all(np.diff(finite) > 0)                  # codes 0..126 ascend
+
+
+def test_every_finite_code_rounds_to_itself():
+    vals = fp8.e4m3_values()
+    finite = vals[~np.isnan(vals)]
+    assert np.array_equal(fp8.e4m3_round(finite), finite)
+
+
+def test_ties_go_to_the_even_mantissa():
+    pos = fp8.e4m3_values()[:127]
+    mids = (pos[:-1] + pos[1:]) / 2
+    r = fp8.e4m3_round(mids)
+    idx = np.searchsorted(pos, r)
+    assert np.all(idx % 2 == 0)
+    assert fp8.e4m3_round(1.0625) == 1.0 and fp8.e4m3_round(1.1875) == 1.25
+
+
+def test_matches_torch_float8_below_saturation():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(0)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.1, 1, 30, 200)])
+    x = x[np.abs(x) < 464].astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    assert np.array_equal(fp8.e4m3_round(x), ref)
+
+
+def test_saturates_and_keeps_nan():
+    r = fp8.e4m3_round(np.array([463.9, 464.0, 1e9, -1e9, np.nan]))
+    assert list(r[:4]) == [448.0, 448.0, 448.0, -448.0] and np.isnan(r[4])
+
+
+def test_relative_error_bound_in_the_normal_range():
+    x = np.geomspace(2.0 ** -6, 440.0, 100000)
+    r = fp8.e4m3_round(x)
+    assert np.max(np.abs(r / x - 1)) <= 2.0 ** -4 + 1e-15
+
+
+def test_block_quantization():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((300, 2, 64)).astype(np.float32)
+    x[128:256, 1] = 0.0                                  # one all-zero block
+    codes, scales = fp8.quantize_blocks(x)
+    assert scales.shape == (3, 2) and scales[1, 1] == 0.0
+    assert np.abs(codes).max() <= 448.0
+    for b in range(3):
+        for h in range(2):
+            blk = codes[b * 128:(b + 1) * 128, h]
+            if scales[b, h] > 0:
+                assert np.abs(blk).max() == 448.0          # the amax element maps to the top code
+    y = fp8.dequantize_blocks(codes, scales)
+    err = np.abs(y - x)
+    bound = np.repeat(scales.astype(np.float64), 128, axis=0)[:300][:, :, None]
+    # half a step of the coarsest binade (2^-4 relative at 448) or a subnormal half-step
+    assert np.all(err <= np.maximum(np.abs(x) * 2.0 ** -4, bound * 2.0 ** -10) + 1e-12)
+
+
+def test_exactly_representable_blocks_give_plain_attention():
+    """Blocks of e4m3 values whose amax is 448 have scale 1 and codes equal to the
+    inputs, so the low-precision attention is the plain attention exactly."""
+    rng = np.random.default_rng(2)
+    pos = fp8.e4m3_values()[:127]
+    def draw(shape):
+        v = rng.choice(pos, size=shape) * rng.choice([-1.0, 1.0], size=shape)
+        v[0::128, :, 0] = 448.0
+        return v.astype(np.float32)
+    q, k = draw((200, 2, 16)), draw((260, 2, 16))
+    v = rng.standard_normal((260, 2, 16))
+    o1, l1 = fp8.attention_fp8_qk(q, k, v, 1e-3)
+    o2, l2 = attention(q, k, v, 1e-3)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_low_precision_attention_is_close_to_exact():
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((256, 2, 128)).astype(np.float32) for _ in range(3))
+    o1, _ = fp8.attention_fp8_qk(q, k, v, 1 / math.sqrt(128))
+    o2, _ = attention(q, k, v, 1 / math.sqrt(128))
+    rel = np.linalg.norm(o1 - o2) / np.linalg.norm(o2)
+    assert 1e-4 < rel < 0.1
