@@ -93,3 +93,28 @@ def test_full_size_832x464_with_four_aux_frames():
         assert np.abs(got["lses"][i] - ref.lses[i]).max() <= TOL_LSE
     assert got["slot_maps"] == ref.slot_maps
     assert ref.n_keys[5] == 27144 + 4 * spec.tokens_per_frame
+
+
+def test_static_scratch_entry_reads_the_aux_frames():
+    """The allocation-free entry point reads the same visible slots (auxiliary ones
+    included) as chunk_attention_fwd: bit-identical outputs."""
+    import torch
+    from kv_cache_chunk_ring_b200 import kvcr
+    spec = wl.shrink(wl.VIDEO_832x464, grid_h=8, grid_w=16, heads=2, chunk_frames=2, sinks=1,
+                     window=2, n_chunks=4, seed=54)
+    T, F = spec.tokens_per_frame, spec.chunk_frames
+    items = list(wl.rollout_chunks(spec))
+    cache = kvcr.Cache(spec.sinks, spec.window, T, spec.heads, spec.head_dim, F,
+                       rope=spec.rope(), aux_frames=3)
+    for it in items[:3]:
+        cache.append(to_dev(it["k"], "bf16"), to_dev(it["v"], "bf16"), it["frames"])
+    k_aux, v_aux, pos = wl.aux_frames(spec, 3, 3)
+    cache.set_aux(to_dev(k_aux, "bf16"), to_dev(v_aux, "bf16"), pos)
+    it = items[3]
+    q, k, v = (to_dev(it[x], "bf16") for x in ("q", "k", "v"))
+    o1, l1 = cache.attention(q, k, v, it["frames"], want_lse=True)
+    o2 = torch.empty_like(q)
+    l2 = torch.empty_like(l1)
+    kvcr.chunk_attention_fwd_static_scratch(cache.handle, q, k, v, it["frames"], o2, l2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

@@ -175,3 +175,25 @@ def test_full_size_sampled():
         assert np.linalg.norm(sum_dk[h]) <= 1e-2 * nk, (h, np.linalg.norm(sum_dk[h]), nk)
         assert np.linalg.norm(sum_dv[h] - sum_do[h]) <= bound_v, \
             (h, np.linalg.norm(sum_dv[h] - sum_do[h]), bound_v)
+
+
+def test_mid_size_head_dim_64_sampled():
+    """4 + 4 chunks of 1000 tokens + a 2-chunk bidirectional block (10000 tokens), 4 heads of
+    head_dim 64: dQ on sampled rows, dK / dV on sampled keys of three block kinds."""
+    spec = wl.MobaSpec("t", heads=4, head_dim=64, n_chunks=4, chunk_tokens=1000,
+                       n_bidir_chunks=2, seed=73)
+    c, L = spec.chunk_tokens, spec.seq_len
+    nc = spec.n_chunks * c
+    (q, k, v, do), _, (dq, dk, dv) = _gpu_fwd_bwd(spec)
+    lay = MobaLayout(spec.n_chunks, c, spec.n_bidir_chunks)
+    scale = 1 / math.sqrt(64)
+    rows = wl.sample_rows(L, 128, 1040, [0, c - 1, c, nc, nc + c - 1, 2 * nc, L - 1])
+    keys = np.array(sorted({3 * c + 5, 3 * c + 999, nc + 2 * c + 7, 2 * nc + 11, L - 1, 0, 130}))
+    import torch
+    ridx = torch.from_numpy(rows).cuda()
+    kidx = torch.from_numpy(keys).cuda()
+    assert_grad_close(to_np(dq.index_select(0, ridx)),
+                      mb.moba_dq_rows(q, k, v, do, lay, rows, scale), "dq d64")
+    ref_dk, ref_dv = mb.moba_dkdv_keys(q, k, v, do, lay, keys, scale)
+    assert_grad_close(to_np(dk.index_select(0, kidx)), ref_dk, "dk d64")
+    assert_grad_close(to_np(dv.index_select(0, kidx)), ref_dv, "dv d64")
