@@ -122,3 +122,69 @@ def test_moba_mutation_caught(monkeypatch):
         return bad_allowed(pos[:, None], pos[None, :], lay)
     monkeypatch.setattr(t_moba, "moba_mask", bad_mask)
     _fails(t_moba.test_rule_table)
+
+
+# ------------------------------------------------ auxiliary frames, fp8, backward
+import importlib                          # noqa: E402
+
+oroll = importlib.import_module("oracle.rollout")   # the package also exports a function of that name
+ofp8 = importlib.import_module("oracle.fp8")
+obwd = importlib.import_module("oracle.moba_bwd")
+from tests import test_oracle_aux as t_aux          # noqa: E402
+from tests import test_oracle_fp8 as t_fp8          # noqa: E402
+from tests import test_oracle_moba_bwd as t_bwd     # noqa: E402
+
+
+def test_aux_keys_left_unrotated_is_caught(monkeypatch):
+    """Auxiliary K used raw although positions were given: the key-duplication pin fails."""
+    real = oroll.rope3d
+    calls = {"n": 0}
+
+    def skip_aux_rotation(x, t, h, w, pairs, base=10000.0):
+        # the rollout rotates Q, K of the chunk (2 calls) and then the auxiliary K
+        calls["n"] += 1
+        if calls["n"] % 3 == 0:
+            return np.asarray(x, dtype=np.float64)
+        return real(x, t, h, w, pairs, base)
+    monkeypatch.setattr(oroll, "rope3d", skip_aux_rotation)
+    _fails(t_aux.test_copies_of_every_visible_frame_double_each_key)
+
+
+def test_fp8_ties_away_from_zero_is_caught(monkeypatch):
+    real_pos = ofp8._POS
+
+    def ties_away(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.abs(x)
+        i = np.clip(np.searchsorted(real_pos, a, side="left"), 1, real_pos.size - 1)
+        lo, hi = real_pos[i - 1], real_pos[i]
+        r = np.where(hi - a <= a - lo, hi, lo)            # ties up instead of to even
+        r = np.where(a >= real_pos[-1], 448.0, r)
+        return np.copysign(np.where(a <= 0, 0.0, r), x)
+    monkeypatch.setattr(ofp8, "e4m3_round", ties_away)
+    _fails(t_fp8.test_ties_go_to_the_even_mantissa)
+
+
+def test_fp8_one_scale_per_tensor_is_caught(monkeypatch):
+    """One amax for the whole tensor (per head) instead of one per 128-row block."""
+    def per_tensor(x, rows=128):
+        x = np.asarray(x, dtype=np.float32)
+        nb = (x.shape[0] + rows - 1) // rows
+        amax = np.abs(x).max(axis=(0, 2)).astype(np.float32)
+        codes = np.zeros(x.shape)
+        for h in range(x.shape[1]):
+            inv = np.float32(448.0) / amax[h]
+            codes[:, h] = ofp8.e4m3_round((x[:, h] * inv).astype(np.float32))
+        return codes, np.tile(amax / np.float32(448.0), (nb, 1))
+    monkeypatch.setattr(ofp8, "quantize_blocks", per_tensor)
+    _fails(t_fp8.test_block_quantization)
+
+
+def test_bwd_missing_scale_on_dk_is_caught(monkeypatch):
+    real = obwd.attention_bwd_masked
+
+    def no_scale_dk(q, k, v, do, allowed, scale):
+        dq, dk, dv = real(q, k, v, do, allowed, scale)
+        return dq, dk / scale, dv
+    monkeypatch.setattr(obwd, "attention_bwd_masked", no_scale_dk)
+    _fails(t_bwd.test_matches_central_finite_differences, 2, 3, 1)
