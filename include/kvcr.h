@@ -144,7 +144,8 @@ int kv_cache_init_aux(kvcr_cache **out, int sinks, int window, int aux_frames,
 int kv_cache_set_aux(kvcr_cache *c, const void *k, const void *v, const int32_t *aux_pos,
                      int n_frames, void *stream);
 
-/* Number of auxiliary frames the next attention call reads. */
+/* Number of auxiliary frames the next attention call reads (0 after the chunk's
+ * append; see kv_cache_set_aux).  Host only; KVCR_EINVAL for NULL arguments. */
 int kv_cache_num_aux(const kvcr_cache *c, int *n);
 
 /* Append finalized frames (the last denoising step's K and V); this finalizes the
@@ -161,7 +162,10 @@ int kv_cache_append_rope(kvcr_cache *c, const void *k, const void *v,
                          const int32_t *frame_idx, int n_frames, void *stream);
 
 /* kv_cache_append_rope() of the same frames into several caches (e.g. every
- * layer's cache at the end of a chunk) in one launch.  caches: host array of
+ * layer's cache at the end of a chunk) in one launch.  The slot rules are those
+ * of kv_cache_append_rope(); batching the layers follows the launch-count
+ * reduction of kaarelkaarelson.com/lingbot (step table: ~20 000 -> ~4 800
+ * launches per chunk).  caches: host array of
  * n_caches distinct handles with the same tokens_per_frame, heads, head_dim,
  * dtype and RoPE (and all with storage, or all bookkeeping-only); k[i], v[i]:
  * device [n_frames * tokens_per_frame][heads][head_dim] for cache i (host
