@@ -222,11 +222,11 @@ int chunk_attention_fwd(kvcr_cache *c, const void *q, int n_q, const void *k_cur
                         float softmax_scale, void *o, float *lse, void *stream);
 
 /* chunk_attention_fwd() for callers that cannot allocate device memory at the
- * time of the call -- for example code that runs while a stream is being
- * captured into a CUDA graph, real-time loops that cannot afford the implicit
- * synchronisation of cudaMalloc/cudaFree, or hosts whose memory pool gives the
- * library exactly the cache buffer.  (The pages describe no such call; it is a
- * property of this library.)  Arguments, result and errors are those of
+ * time of the call: hosts whose memory pool owns every device allocation and
+ * hands the library exactly the cache buffer, and real-time loops that cannot
+ * take the implicit device synchronisation of cudaMalloc/cudaFree.  (The
+ * papers have no counterpart of this call; it is a property of this library.)
+ * Arguments, result and errors are those of
  * chunk_attention_fwd().  The difference: the rotated queries and current-chunk
  * keys are staged in a fixed 36 MiB array that the library holds in device
  * memory on every GPU where it is loaded (until the process exits), not in the

@@ -1,12 +1,11 @@
 // Library-owned staging memory for chunk_attention_fwd_static_scratch().
 //
 // Some callers cannot allocate device memory when they call into the
-// library: code running while a stream is being captured into a CUDA graph
-// (where an allocation call would break the capture), real-time loops that
-// must not take the implicit device synchronisation of cudaMalloc/cudaFree,
-// and hosts whose memory pool hands out exactly the cache buffer and nothing
-// more.  For them the rotated queries and current-chunk keys of one chunk are
-// staged in this fixed file-scope array instead of a caller buffer.
+// library: hosts whose memory pool owns every allocation and hands out exactly
+// the cache buffer and nothing more, and real-time loops that must not take
+// the implicit device synchronisation of cudaMalloc/cudaFree.  For them the
+// rotated queries and current-chunk keys of one chunk are staged in this fixed
+// file-scope array instead of a caller buffer.
 //
 // The array is kStaticScratchBytes (36 MiB) and lives on every GPU on which
 // this module is loaded, until the process exits.  All calls on a device share

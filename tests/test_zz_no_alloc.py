@@ -1,11 +1,11 @@
 """chunk_attention_fwd_static_scratch: chunk attention that allocates nothing.
 
 It exists for callers that cannot allocate device memory when they call the
-library -- code that runs while a stream is being captured into a CUDA graph,
-real-time loops that cannot take the device synchronisation of
-cudaMalloc/cudaFree, or hosts whose memory pool hands the library only the
-cache buffer.  Instead of the cache's scratch region it stages the rotated
-queries and keys in a fixed 36 MiB array the library keeps on the device.
+library -- hosts whose memory pool owns every allocation and hands the library
+only the cache buffer, or real-time loops that cannot take the device
+synchronisation of cudaMalloc/cudaFree.  Instead of the cache's scratch region
+it stages the rotated queries and keys in a fixed 36 MiB array the library
+keeps on the device.
 
 These tests call it through the C ABI and check, on two calls in a row per
 chunk, that it returns what chunk_attention_fwd returns (same tolerances as
