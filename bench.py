@@ -10,9 +10,15 @@ non-anchor frames evicted).  The metric is useful attention TFLOP/s
 the dense bf16 roofline and the append kernel's GB/s reported beside it.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
-layer cache (weak scaling, no collective on the data path); the timed region
-is bracketed by barriers and the max elapsed time over ranks is reported.
+                [--shard heads|layers]
+Multi-GPU (one process per GPU; ``--gpus N`` without torchrun starts the N ranks
+through torch.distributed.run): with ``--shard heads`` (the default) rank r owns
+a contiguous range of the 12 heads of the layer cache, so the ranks split one
+chunk step (strong scaling); with ``--shard layers`` every rank runs a layer
+cache of its own (weak scaling).  Neither has a collective on the data path;
+the timed region is bracketed by barriers and the max elapsed time over ranks
+is reported.  At one GPU the line also carries the 30-layer x 4-step chunk
+(120 attention calls and one batched append of 30 layer caches) as extra keys.
 ``--impl reference`` times the CPU oracle on a bounded sample of the same
 workload (rank 0 only).
 """
@@ -36,6 +42,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+from kv_cache_chunk_ring_b200 import shard as sh  # noqa: E402
 from kv_cache_chunk_ring_b200 import workloads as wl  # noqa: E402
 
 SPEC = wl.VIDEO_832x464
@@ -46,18 +53,18 @@ POOL = 3                  # distinct input chunks cycled through the timed steps
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def step_flops(spec=SPEC) -> float:
+def step_flops(spec=SPEC, heads=None) -> float:
     lq = spec.chunk_tokens
     lk = (spec.sinks + spec.window + spec.chunk_frames) * spec.tokens_per_frame
-    return 4.0 * lq * lk * spec.heads * spec.head_dim
+    return 4.0 * lq * lk * (spec.heads if heads is None else heads) * spec.head_dim
 
 
-def append_bytes(spec=SPEC) -> float:
+def append_bytes(spec=SPEC, heads=None) -> float:
     # read K and V, write rotated K and V: 4 * F * T * H * D * 2 bytes
-    return 4.0 * spec.chunk_tokens * spec.heads * spec.head_dim * 2
+    return 4.0 * spec.chunk_tokens * (spec.heads if heads is None else heads) * spec.head_dim * 2
 
 
-def config_dict(spec=SPEC) -> dict:
+def config_dict(spec=SPEC, shard="heads", world=1) -> dict:
     lk = (spec.sinks + spec.window + spec.chunk_frames) * spec.tokens_per_frame
     return {
         "workload": spec.name,
@@ -67,6 +74,8 @@ def config_dict(spec=SPEC) -> dict:
         "q_tokens": spec.chunk_tokens, "keys": lk,
         "step": "chunk_attention_fwd (RoPE stage + attention) + kv_cache_append_rope, steady state",
         "l2": "inputs larger than L2: each step reads 130 MB of cached K/V + 55.6 MB chunk inputs",
+        "parallelism": ("single GPU" if world == 1 else
+                        f"{world} ranks, {'heads of one layer cache split' if shard == 'heads' else 'one layer cache each'}; no collective"),
     }
 
 
@@ -79,30 +88,29 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+ATTN_SOURCES = ("attn_sm100.cu", "sm100_ptx.cuh", "kvcr_internal.h")
+
+
+def kernel_source_hash(names=ATTN_SOURCES) -> str:
     h = hashlib.sha256()
-    for name in ("attn_sm100.cu", "sm100_ptx.cuh", "kvcr_internal.h"):
+    for name in names:
         with open(os.path.join(ROOT, "kv_cache_chunk_ring_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic():
-    """DRAM bytes per launch of the attention kernel from the committed ncu summary,
-    or None when that summary is missing or was taken on different kernel source."""
-    p = os.path.join(ROOT, "profiles", "chunk_attn_832x464_ncu.md")
+def recorded_traffic(record="chunk_attn_832x464.json", names=ATTN_SOURCES):
+    """DRAM bytes per launch of a kernel from its committed ncu record (JSON: source
+    hash and dram bytes per launch), or None when the record is missing or was taken
+    on different kernel source."""
+    p = os.path.join(ROOT, "profiles", record)
     if not os.path.exists(p):
         return None
-    src = None
-    traffic = None
-    for line in open(p):
-        if line.startswith("source-hash:"):
-            src = line.split(":", 1)[1].strip()
-        if line.startswith("dram-bytes-per-launch:"):
-            traffic = float(line.split(":", 1)[1].strip())
-    if src != kernel_source_hash():
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("source_hash") != kernel_source_hash(names):
         return None
-    return traffic
+    return float(rec["dram_bytes_per_launch"])
 
 
 class ClockSampler:
@@ -161,6 +169,15 @@ class ClockSampler:
 
 # ---------------------------------------------------------- multi-process --
 
+def free_port() -> int:
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
 def max_over_ranks(value: float, dist, device) -> float:
     """The largest of every rank's value (the whole job ends when the slowest rank does)."""
     if dist is None:
@@ -190,15 +207,22 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     spec = SPEC
-    T, H, D, F = spec.tokens_per_frame, spec.heads, spec.head_dim, spec.chunk_frames
+    shard = args.shard if world > 1 else "heads"
+    if shard == "heads":                    # this rank's heads of the one layer cache
+        h0, h1 = sh.head_range(spec.heads, world, rank)
+        layer = 0
+    else:                                   # a layer cache of its own, all heads
+        h0, h1 = 0, spec.heads
+        layer = rank
+    T, H, D, F = spec.tokens_per_frame, h1 - h0, spec.head_dim, spec.chunk_frames
     stream = torch.cuda.current_stream()
 
     cache = kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope())
-    # seeded synthetic chunks (each rank its own layer seed): fill chunks + a pool for timing
-    gen = wl.rollout_chunks(wl.shrink(spec, n_chunks=STEADY_CHUNK + POOL), layer=rank)
+    # seeded synthetic chunks: fill chunks + a pool for timing, this rank's heads
+    gen = wl.rollout_chunks(wl.shrink(spec, n_chunks=STEADY_CHUNK + POOL), layer=layer)
     chunks = []
     for item in gen:
-        chunks.append(tuple(torch.from_numpy(item[x]).to(dev, torch.bfloat16)
+        chunks.append(tuple(sh.slice_heads(torch.from_numpy(item[x]), h0, h1).to(dev, torch.bfloat16)
                             for x in ("q", "k", "v")))
     o = torch.empty_like(chunks[0][0])
     frame = [0]
@@ -309,23 +333,26 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     kvcr.kvcr_check_status()
 
-    flops = step_flops(spec)
-    value = whole_job_throughput(world, args.steps, flops, elapsed_ms)
-    e2e_value = whole_job_throughput(world, args.steps, flops, e2e_ms)
+    flops = step_flops(spec, H)                     # this rank's work per step
+    # the whole job per step: one 12-head layer split by head, or one layer per rank
+    job_ranks = 1 if shard == "heads" else world
+    value = whole_job_throughput(job_ranks, args.steps, step_flops(spec), elapsed_ms)
+    e2e_value = whole_job_throughput(job_ranks, args.steps, step_flops(spec), e2e_ms)
     peaks, peak_kind = load_peaks()
     attn = kt.get("chunk_attn", {})
     attn_ms = attn.get("avg_ms", float("nan"))
     achieved = flops / (attn_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     app = kt.get("append_rope", {})
-    app_gbs = append_bytes(spec) / (app.get("avg_ms", float("nan")) * 1e-3) / 1e9
-    chunk_bytes = spec.chunk_tokens * H * D * 2
+    app_gbs = append_bytes(spec, H) / (app.get("avg_ms", float("nan")) * 1e-3) / 1e9
+    chunk_bytes = job_ranks * spec.chunk_tokens * spec.heads * D * 2   # whole job
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_dict(spec),
+        "scaling": "strong" if (shard == "heads" and world > 1) else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(spec, shard, world),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": recorded_traffic(),
@@ -477,8 +504,9 @@ def _timed(fn, steps, warmup):
     return e0.elapsed_time(e1) / steps
 
 
-def run_layers30(args) -> dict:
-    """30 layers x 4 denoising steps per chunk (120 attention calls + 30 appends)."""
+def run_layers30(args, clocks=False) -> dict:
+    """30 layers x 4 denoising steps per chunk (120 attention calls + 30 appends), timed
+    with one append per layer and with one batched append of the 30 caches."""
     import torch
     from kv_cache_chunk_ring_b200 import build as _build
     from kv_cache_chunk_ring_b200 import kvcr
@@ -520,8 +548,12 @@ def run_layers30(args) -> dict:
     for _ in range(STEADY_CHUNK):
         chunk()
     kvcr.kvcr_trace_reset()
+    sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if sampler:
+        sampler.start()
     ms = _timed(chunk, args.steps, args.warmup)
     ms_batched = _timed(chunk_batched, args.steps, args.warmup)
+    clk = sampler.stop() if sampler else None
     kvcr.kvcr_trace_enable(True)
     chunk()
     chunk_batched()
@@ -532,7 +564,14 @@ def run_layers30(args) -> dict:
     flops = spec.layers * spec.steps * step_flops(spec)
     bat_n, bat_ms = kt["append_batch"]
     app_n, app_ms = kt["append_rope"]
+    peaks, _ = load_peaks()
+    attn_call_ms = kt["chunk_attn"][1] / max(1, kt["chunk_attn"][0])
+    bat_gbs = spec.layers * append_bytes(spec) / (bat_ms / max(1, bat_n) * 1e-3) / 1e9
     return {"workload": spec.name, "ms_per_chunk": round(ms, 3),
+            "attn_kernel_frac": round(step_flops(spec) / (attn_call_ms * 1e-3) / 1e12 /
+                                      float(peaks["bf16_tflops"]), 4),
+            "append_batch_hbm_frac": round(bat_gbs / float(peaks["hbm_gbs"]), 4),
+            "clocks": clk,
             "attention_tflops_per_chunk": round(flops / 1e12, 2),
             "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": UNIT,
             "attn_kernel_ms": round(kt["chunk_attn"][1] / max(1, kt["chunk_attn"][0]), 4),
@@ -758,6 +797,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-layers30", action="store_true",
+                    help="leave out the 30-layer chunk figures of the default line")
+    ap.add_argument("--shard", default="heads", choices=["heads", "layers"],
+                    help="multi-GPU partition: heads of one layer cache per rank (strong "
+                         "scaling) or one layer cache per rank (weak scaling)")
     ap.add_argument("--moba-chunk-tokens", type=int, default=0,
                     help="moba_bwd: tokens per chunk (default: the workload's 6032); a smaller "
                          "value gives a case small enough for a full profiler capture")
@@ -769,6 +813,14 @@ def main():
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # start one rank per GPU through torch.distributed.run, with the same arguments
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+               f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+               f"--master-port={free_port()}", os.path.abspath(__file__)] + sys.argv[1:]
+        sys.exit(subprocess.call(cmd))
+    if world > 1 and args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but {world} ranks were started")
 
     if args.impl == "reference":
         if rank == 0:
@@ -793,6 +845,24 @@ def main():
     try:
         out = run_ours(args, rank, world, dist)
         if rank == 0:
+            if world == 1 and not args.no_layers30:
+                # the 30-layer x 4-step chunk (each layer its own cache, 5 GB: no reuse of
+                # one call's K/V by the next in L2), measured after the timed region
+                l30 = run_layers30(argparse.Namespace(steps=max(3, min(args.steps, 10)),
+                                                      warmup=3), clocks=True)
+                out.update({
+                    "layers30_ms_per_chunk": l30["ms_per_chunk_batched_append"],
+                    "layers30_ms_per_chunk_separate_appends": l30["ms_per_chunk"],
+                    "layers30_attn_kernel_ms": l30["attn_kernel_ms"],
+                    "layers30_attn_kernel_frac": l30["attn_kernel_frac"],
+                    "layers30_append_gb_s": l30["append_batch_gb_s"],
+                    "layers30_append_hbm_frac": l30["append_batch_hbm_frac"],
+                    "layers30_append_separate_gb_s": l30["append_gb_s"],
+                    "layers30_clocks": l30["clocks"],
+                    "layers30_note": "30 layer caches x 4 denoising steps per chunk: 120 "
+                                     "attention calls + one batched append of 30 caches "
+                                     "(separate appends timed too); steady-state chunks",
+                })
             if world == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = cpu_baseline()
             print(json.dumps(out))

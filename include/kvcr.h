@@ -36,6 +36,10 @@
  *    caller-owned device buffer of kv_cache_storage_bytes() bytes.
  *  - All compute runs in the library's own CUDA kernels; there is no CPU
  *    fallback.
+ *  - A failure inside a kernel (a bounded wait that ran out) happens after the
+ *    launching call has returned KVCR_OK: poll kvcr_check_status() after the
+ *    stream's work to learn of it; until then the outputs of that work are
+ *    not to be trusted.
  */
 #ifndef KVCR_H
 #define KVCR_H
@@ -90,7 +94,14 @@ typedef struct kvcr_cache kvcr_cache;
 
 /* ---------------------------------------------------------------- cache --- */
 
-/* Bytes of device storage a cache needs: K and V of sinks+window frame slots,
+/* The cache is the per-layer KV store of a chunk-wise causal video stream:
+ * anchor tokens kept at the front plus a sliding window of recent frames
+ * ("LingBot-World-Infinity: The Open-Source World Model That Refuses to
+ * Forget", "How the cache keeps the world alive"; "Westlake AGI Lab's 'World
+ * in World' Steers Frozen Video Models", second paragraph: 6 anchor + 8
+ * recent latent-frame slots).
+ *
+ * Bytes of device storage a cache needs: K and V of sinks+window frame slots,
  * and, when with_rope != 0, scratch for the rotated queries and current-chunk
  * keys of one chunk (chunk_frames frames) plus the (h, w) angle tables.
  * Returns 0 for invalid sizes. */
@@ -149,7 +160,9 @@ int kv_cache_set_aux(kvcr_cache *c, const void *k, const void *v, const int32_t 
 int kv_cache_num_aux(const kvcr_cache *c, int *n);
 
 /* Append finalized frames (the last denoising step's K and V); this finalizes the
- * chunk, so its auxiliary frames (kv_cache_set_aux) are dropped.
+ * chunk, so its auxiliary frames (kv_cache_set_aux) are dropped.  Each generated
+ * chunk's state is appended, the oldest non-anchor state evicted and the anchors
+ * kept ("LingBot-World-Infinity", "The trick: treat video like a causal stream").
  * k, v: device [n_frames * tokens_per_frame][heads][head_dim].  frame_idx: host,
  * n_frames strictly increasing absolute latent-frame indices, each larger than
  * every frame appended before.  Frame by frame: an unfilled anchor slot is taken
@@ -179,21 +192,27 @@ int kv_cache_append_rope_batch(kvcr_cache *const *caches, int n_caches, const vo
                                void *stream);
 
 /* Dynamic window: evict the oldest non-anchor frames until at most keep_recent
- * remain (0 <= keep_recent <= window).  Host only.  evicted_out (nullable) receives
+ * remain (0 <= keep_recent <= window).  Host only.  This is the hook of a
+ * dynamic KV-cache scheduler that adapts the retained history to the current
+ * control signal ("Infinite Worlds with Versatile Interactions", deployment
+ * paragraph).  evicted_out (nullable) receives
  * up to evicted_cap evicted frame indices, oldest first; *n_evicted (nullable)
  * the number evicted. */
 int kv_cache_evict(kvcr_cache *c, int keep_recent, int32_t *evicted_out, int evicted_cap,
                    int *n_evicted);
 
-/* Slot table: frame_of_slot[s] = frame cached in slot s or -1, s < sinks+window. */
+/* Slot table: frame_of_slot[s] = frame cached in slot s or -1, s < sinks+window
+ * (the anchor and recent slots of "World in World", second paragraph); cap =
+ * length of frame_of_slot (>= sinks + window).  Host only. */
 int kv_cache_slot_map(const kvcr_cache *c, int32_t *frame_of_slot, int cap);
 
 /* Result of the last append: slot of each appended frame (-1 = not retained)
- * and the frames it evicted (oldest first). */
+ * and the frames it evicted (oldest first).  A read-back of the slot rules
+ * above; no page has a counterpart (library convention).  Host only. */
 int kv_cache_last_append(const kvcr_cache *c, int32_t *slots, int slots_cap,
                          int32_t *evicted, int evicted_cap, int *n_evicted);
 
-/* Number of cached frames. */
+/* Number of cached frames (library convention; host only). */
 int kv_cache_num_cached(const kvcr_cache *c, int *n);
 
 /* Device addresses of slot `slot`'s K and V, each [tokens_per_frame][heads][head_dim]
@@ -207,7 +226,10 @@ void kv_cache_destroy(kvcr_cache *c);
 
 /* Chunk attention: O = softmax(scale * Q K^T) V where the keys are every cached
  * frame (anchors and window) followed by the current chunk's own n_cur_frames
- * frames; full attention inside the chunk.
+ * frames; full attention inside the chunk.  The block reads the anchor slots,
+ * the recent slots and the current chunk ("Westlake AGI Lab's 'World in World'
+ * Steers Frozen Video Models", second paragraph: 6 + 8 + 4 latent-frame slots;
+ * "LingBot-World-Infinity", "How the cache keeps the world alive").
  *   q:     device [n_q][heads][head_dim]; with RoPE, n_q must equal
  *          n_cur_frames * tokens_per_frame (the chunk's tokens) and Q is rotated
  *          at the chunk's positions; without RoPE n_q is free (cross-attention).
@@ -244,7 +266,10 @@ int chunk_attention_fwd_static_scratch(kvcr_cache *c, const void *q, int n_q,
                                        const int32_t *cur_frame_idx, int n_cur_frames,
                                        float softmax_scale, void *o, float *lse, void *stream);
 
-/* Attention under the MoBA mask over one sequence of L = layout tokens.
+/* Attention under the MoBA mask over one sequence of L = layout tokens ("Infinite
+ * Worlds with Versatile Interactions", causal-pretraining paragraph: the
+ * teacher-forcing mask plus an appended fully bidirectional block; "Mix Forcing",
+ * "Mix the training modes").
  * q, k, v, o: device [L][heads][head_dim] bf16 (head_dim 128 or 64); lse nullable
  * fp32 [heads][L].  128 x 128 tiles of the score matrix with no allowed entry
  * are skipped, fully allowed tiles run unmasked, the rest are masked. */
@@ -284,7 +309,10 @@ int moba_attention_bwd(const void *q, const void *k, const void *v, const void *
 size_t moba_attention_bwd_workspace_bytes(const kvcr_moba_layout *layout, int heads);
 
 /* Host classification of the tile x tile blocks of the MoBA score matrix into
- * KVCR_TILE_EMPTY / PARTIAL / FULL (only in-range rows and columns count).
+ * KVCR_TILE_EMPTY / PARTIAL / FULL (only in-range rows and columns count).  The
+ * pages give the mask, not a tiling: this is the block-sparse schedule of this
+ * library's MoBA kernels (empty tiles skipped, full ones unmasked), exported so
+ * it can be checked against a brute-force reduction of the mask.
  * cls: host [nt * nt] row-major, nt = ceil(L / tile); cap = its length. */
 int moba_classify_tiles(const kvcr_moba_layout *layout, int tile, uint8_t *cls, size_t cap);
 
@@ -292,9 +320,11 @@ int moba_classify_tiles(const kvcr_moba_layout *layout, int tile, uint8_t *cls, 
 
 /* Synchronise `stream` and return (then clear) the device-side status of the
  * library's kernels on the current device: KVCR_OK or KVCR_ETIMEOUT when a
- * kernel gave up on a bounded wait (its outputs are then invalid). */
+ * kernel gave up on a bounded wait (its outputs are then invalid).  Library
+ * convention (failure detection); no page has a counterpart. */
 int kvcr_check_status(void *stream);
 
+/* Message of the last non-OK return on this thread (library convention). */
 const char *kvcr_last_error(void);
 
 /* Failure-path test hook (for tests; off by default).  kind = 1 makes every
@@ -324,7 +354,8 @@ enum {
     KVCR_K_COUNT = 10
 };
 
-/* Count of every kernel the library launched in this process. */
+/* Count of every kernel the library launched in this process (library
+ * convention, for launch accounting). */
 long long kvcr_launch_count(void);
 
 /* Tracing: when on, each launch is bracketed by two CUDA events recorded on

@@ -51,6 +51,93 @@ class KvcrError(RuntimeError):
         self.code = code
 
 
+class KvcrArgError(KvcrError, ValueError):
+    """A tensor argument that does not match what the call reads or writes; raised by
+    the binding before anything reaches the library (nothing is launched)."""
+
+
+# Sizes of every live cache handle (handle value -> (T, H, D, dtype code, has RoPE)), so the
+# tensor-taking calls can check their arguments against the cache before a launch.
+_CACHE_INFO = {}
+
+
+def _expect(specs) -> None:
+    """Raise KvcrArgError unless every (name, tensor, shape, torch dtype) of ``specs`` is a
+    contiguous tensor of exactly that shape and dtype, and all of them are CUDA tensors
+    on one device.  Shapes, dtypes and layouts are checked before devices, so a
+    mismatch is reported the same way on a host without a GPU."""
+    for name, t, shape, dtype in specs:
+        if t is None:
+            raise KvcrArgError(KVCR_EINVAL, f"{name} is required")
+        shape = tuple(int(x) for x in shape)
+        if tuple(t.shape) != shape:
+            raise KvcrArgError(KVCR_ESHAPE, f"{name} has shape {tuple(t.shape)}, expected {shape}")
+        if t.dtype != dtype:
+            raise KvcrArgError(KVCR_EINVAL, f"{name} has dtype {t.dtype}, expected {dtype}")
+        if not t.is_contiguous():
+            raise KvcrArgError(KVCR_EINVAL, f"{name} must be contiguous")
+    device = specs[0][1].device
+    for name, t, _, _ in specs:
+        if not t.is_cuda:
+            raise KvcrArgError(KVCR_EINVAL, f"{name} must be a CUDA tensor")
+        if t.device != device:
+            raise KvcrArgError(KVCR_EINVAL, f"{name} is on {t.device}, {specs[0][0]} on {device}")
+
+
+def _torch_dtype(code: int):
+    import torch
+    return torch.bfloat16 if code == KVCR_BF16 else torch.float32
+
+
+def _cache_info(handle):
+    key = handle.value if isinstance(handle, ctypes.c_void_p) else handle
+    info = _CACHE_INFO.get(key)
+    if info is None:
+        raise KvcrArgError(KVCR_EINVAL, "unknown or destroyed cache handle")
+    return info
+
+
+def _check_chunk_args(handle, q, k_cur, v_cur, n_frames: int, o, lse) -> None:
+    """Tensor arguments of chunk attention against the cache's sizes."""
+    import torch
+    T, H, D, dt, rope = _cache_info(handle)
+    if q is None or q.dim() != 3:
+        raise KvcrArgError(KVCR_ESHAPE, "q must be [n_q, heads, head_dim]")
+    n_q, n_cur = q.shape[0], n_frames * T
+    if rope and n_q != n_cur:
+        raise KvcrArgError(KVCR_ESHAPE, f"q has {n_q} rows; with RoPE it must have "
+                                        f"n_cur_frames * tokens_per_frame = {n_cur}")
+    dt = _torch_dtype(dt)
+    specs = [("q", q, (n_q, H, D), dt), ("k_cur", k_cur, (n_cur, H, D), dt),
+             ("v_cur", v_cur, (n_cur, H, D), dt), ("o", o, (n_q, H, D), dt)]
+    if lse is not None:
+        specs.append(("lse", lse, (H, n_q), torch.float32))
+    _expect(specs)
+
+
+def _check_kv(handle, k, v, n_frames: int, what: str) -> None:
+    T, H, D, dt, _ = _cache_info(handle)
+    if k is None and v is None:
+        return                                   # bookkeeping-only call; the library checks
+    dt = _torch_dtype(dt)
+    _expect([(f"{what} k", k, (n_frames * T, H, D), dt),
+             (f"{what} v", v, (n_frames * T, H, D), dt)])
+
+
+def _check_moba_args(L: int, tensors, lse) -> None:
+    """q, k, v, o (and the backward's tensors) all [L, heads, head_dim] in one dtype and
+    device; lse fp32 [heads, L]."""
+    import torch
+    first = tensors[0][1]
+    if first is None or first.dim() != 3:
+        raise KvcrArgError(KVCR_ESHAPE, f"{tensors[0][0]} must be [L, heads, head_dim]")
+    shape = (L, first.shape[1], first.shape[2])
+    specs = [(name, t, shape, first.dtype) for name, t in tensors]
+    if lse is not None:
+        specs.append(("lse", lse, (shape[1], L), torch.float32))
+    _expect(specs)
+
+
 class kvcr_rope(ctypes.Structure):
     _fields_ = [("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int), ("pairs_t", ctypes.c_int),
                 ("pairs_h", ctypes.c_int), ("pairs_w", ctypes.c_int), ("base", ctypes.c_double)]
@@ -180,11 +267,14 @@ def kv_cache_init_aux(sinks, window, aux_frames, tokens_per_frame, heads, head_d
     _check(lib().kv_cache_init_aux(ctypes.byref(h), sinks, window, aux_frames, tokens_per_frame,
                                    heads, head_dim, chunk_frames, rp, _dtype_code(dtype), ptr,
                                    nbytes))
+    _CACHE_INFO[h.value] = (tokens_per_frame, heads, head_dim, _dtype_code(dtype),
+                            rope is not None)
     return h
 
 
 def kv_cache_set_aux(handle, k, v, aux_pos: Optional[Sequence[int]], n_frames: int,
                      stream=None) -> None:
+    _check_kv(handle, k, v, n_frames, "kv_cache_set_aux")
     s = None if (k is None and v is None) else _stream(stream)
     pos = None if aux_pos is None else _i32(aux_pos)
     _check(lib().kv_cache_set_aux(handle, _ptr(k), _ptr(v), pos, n_frames, s))
@@ -208,11 +298,14 @@ def kv_cache_init(sinks, window, tokens_per_frame, heads, head_dim, chunk_frames
     nbytes = 0 if storage is None else storage.numel() * storage.element_size()
     _check(lib().kv_cache_init(ctypes.byref(h), sinks, window, tokens_per_frame, heads, head_dim,
                                chunk_frames, rp, _dtype_code(dtype), ptr, nbytes))
+    _CACHE_INFO[h.value] = (tokens_per_frame, heads, head_dim, _dtype_code(dtype),
+                            rope is not None)
     return h
 
 
 def kv_cache_append_rope(handle, k, v, frame_idx: Sequence[int], stream=None) -> None:
     n = len(frame_idx)
+    _check_kv(handle, k, v, n, "kv_cache_append_rope")
     s = None if (k is None and v is None) else _stream(stream)
     _check(lib().kv_cache_append_rope(handle, _ptr(k), _ptr(v), _i32(frame_idx), n, s))
 
@@ -226,6 +319,15 @@ def kv_cache_append_rope_batch(handles, ks, vs, frame_idx: Sequence[int], stream
         kp = vp = None
         s = None
     else:
+        if len(ks) != n or len(vs) != n:
+            raise KvcrArgError(KVCR_ESHAPE, "one k and one v per cache")
+        specs = []
+        for i, h in enumerate(handles):
+            T, H, D, dt, _ = _cache_info(h)
+            shape = (len(frame_idx) * T, H, D)
+            specs += [(f"kv_cache_append_rope_batch[{i}] k", ks[i], shape, _torch_dtype(dt)),
+                      (f"kv_cache_append_rope_batch[{i}] v", vs[i], shape, _torch_dtype(dt))]
+        _expect(specs)
         kp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in ks])
         vp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in vs])
         s = _stream(stream)
@@ -273,11 +375,13 @@ def kv_cache_slot_data(handle, slot: int) -> Tuple[int, int]:
 
 
 def kv_cache_destroy(handle) -> None:
+    _CACHE_INFO.pop(handle.value if isinstance(handle, ctypes.c_void_p) else handle, None)
     lib().kv_cache_destroy(handle)
 
 
 def chunk_attention_fwd(handle, q, k_cur, v_cur, cur_frame_idx: Sequence[int], o, lse=None,
                         softmax_scale: float = 0.0, stream=None) -> None:
+    _check_chunk_args(handle, q, k_cur, v_cur, len(cur_frame_idx), o, lse)
     _check(lib().chunk_attention_fwd(handle, _ptr(q), q.shape[0], _ptr(k_cur), _ptr(v_cur),
                                      _i32(cur_frame_idx), len(cur_frame_idx),
                                      float(softmax_scale), _ptr(o), _ptr(lse), _stream(stream)))
@@ -287,6 +391,7 @@ def chunk_attention_fwd_static_scratch(handle, q, k_cur, v_cur, cur_frame_idx: S
                                        lse=None, softmax_scale: float = 0.0,
                                        stream=None) -> None:
     """chunk_attention_fwd staged in the library's fixed device array (allocates nothing)."""
+    _check_chunk_args(handle, q, k_cur, v_cur, len(cur_frame_idx), o, lse)
     _check(lib().chunk_attention_fwd_static_scratch(
         handle, _ptr(q), q.shape[0], _ptr(k_cur), _ptr(v_cur), _i32(cur_frame_idx),
         len(cur_frame_idx), float(softmax_scale), _ptr(o), _ptr(lse), _stream(stream)))
@@ -294,6 +399,8 @@ def chunk_attention_fwd_static_scratch(handle, q, k_cur, v_cur, cur_frame_idx: S
 
 def moba_attention_fwd(q, k, v, n_chunks: int, chunk_tokens: int, n_bidir_chunks: int, o,
                        lse=None, softmax_scale: float = 0.0, stream=None) -> None:
+    L = (2 * n_chunks + n_bidir_chunks) * chunk_tokens
+    _check_moba_args(L, [("q", q), ("k", k), ("v", v), ("o", o)], lse)
     lay = kvcr_moba_layout(n_chunks, chunk_tokens, n_bidir_chunks)
     _check(lib().moba_attention_fwd(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(lay), q.shape[1],
                                     q.shape[2], _dtype_code(q.dtype), float(softmax_scale),
@@ -312,11 +419,18 @@ def moba_attention_bwd(q, k, v, o, d_o, lse, n_chunks: int, chunk_tokens: int,
     """dQ, dK, dV of moba_attention_fwd into dq, dk, dv.  ``workspace`` is a device
     tensor of at least moba_attention_bwd_workspace_bytes() bytes (allocated here
     with torch when omitted)."""
+    L = (2 * n_chunks + n_bidir_chunks) * chunk_tokens
+    if lse is None:
+        raise KvcrArgError(KVCR_EINVAL, "lse (the forward's) is required")
+    _check_moba_args(L, [("q", q), ("k", k), ("v", v), ("o", o), ("d_o", d_o), ("dq", dq),
+                         ("dk", dk), ("dv", dv)], lse)
     lay = kvcr_moba_layout(n_chunks, chunk_tokens, n_bidir_chunks)
     need = int(lib().moba_attention_bwd_workspace_bytes(ctypes.byref(lay), q.shape[1]))
     if workspace is None:
         import torch
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or workspace.device != q.device or not workspace.is_contiguous():
+        raise KvcrArgError(KVCR_EINVAL, "workspace must be a contiguous tensor on q's device")
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib().moba_attention_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), ctypes.byref(lay),

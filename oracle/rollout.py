@@ -41,7 +41,7 @@ import numpy as np
 
 from .attn import attention
 from .cache import CacheModel
-from .rope import rope3d, rope_positions
+from .rope import rope3d, rope_pairs_default, rope_positions
 
 
 @dataclasses.dataclass
@@ -69,6 +69,10 @@ def rollout(spec, chunks, rows_for=None, use_rope: bool = True,
     T = spec.grid_h * spec.grid_w
     scale = 1.0 / math.sqrt(spec.head_dim)
     pairs = (spec.rope().pairs_t, spec.rope().pairs_h, spec.rope().pairs_w)
+    # the workload states the split; it must be the oracle's own pinned default
+    if pairs != rope_pairs_default(spec.head_dim):
+        raise ValueError(f"RoPE pair split {pairs} differs from the oracle's default "
+                         f"{rope_pairs_default(spec.head_dim)} for head_dim {spec.head_dim}")
     cap = spec.window if window_schedule is None else max(spec.window, max(window_schedule))
     cache = CacheModel(spec.sinks, cap)
     store: Dict[int, tuple] = {}     # frame -> (K_rot [T,H,D], V [T,H,D])

@@ -111,3 +111,52 @@ def test_clean_chunks_causal():
 def test_allowed_broadcast_shapes():
     lay = MobaLayout(2, 3, 1)
     assert moba_allowed(np.arange(15)[:, None], np.arange(15)[None, :], lay).shape == (15, 15)
+
+
+def _tile_counts_by_intervals(n, c, mb, tile=128):
+    """Independent count of the tile classes: each query row's readable keys written
+    as at most two intervals straight from the rule (C_i: [0, (i+1)c); N_i:
+    [0, i c) and [nc + i c, nc + (i+1) c); B: [2nc, L)), overlapped with every key
+    tile and summed over the rows of each query tile."""
+    nc = n * c
+    L = (2 * n + mb) * c
+    nt = (L + tile - 1) // tile
+    kt0 = np.arange(nt) * tile
+    kt1 = np.minimum(kt0 + tile, L)
+    counts = {TILE_FULL: 0, TILE_PARTIAL: 0, TILE_EMPTY: 0}
+    for qt in range(nt):
+        r = np.arange(qt * tile, min((qt + 1) * tile, L))
+        i = np.where(r < nc, r // c, np.where(r < 2 * nc, (r - nc) // c, 0))
+        lo0 = np.where(r < 2 * nc, 0, 2 * nc)
+        hi0 = np.where(r < nc, (i + 1) * c, np.where(r < 2 * nc, i * c, L))
+        lo1 = np.where((r >= nc) & (r < 2 * nc), nc + i * c, 0)
+        hi1 = np.where((r >= nc) & (r < 2 * nc), nc + (i + 1) * c, 0)
+        ov = np.zeros(nt, dtype=np.int64)
+        for lo, hi in ((lo0, hi0), (lo1, hi1)):
+            a = np.clip(np.minimum(hi[:, None], kt1[None, :]) - np.maximum(lo[:, None], kt0[None, :]),
+                        0, None)
+            ov += a.sum(axis=0)
+        area = r.size * (kt1 - kt0)
+        counts[TILE_FULL] += int((ov == area).sum())
+        counts[TILE_EMPTY] += int((ov == 0).sum())
+        counts[TILE_PARTIAL] += int(((ov > 0) & (ov < area)).sum())
+    return counts
+
+
+@pytest.mark.parametrize("n,c,mb,tile", [(3, 7, 2, 4), (5, 6, 3, 4), (2, 16, 2, 16), (3, 50, 2, 128)])
+def test_tile_counts_by_intervals_small(n, c, mb, tile):
+    ref = classify_tiles_mask(MobaLayout(n, c, mb), tile)
+    got = _tile_counts_by_intervals(n, c, mb, tile)
+    assert got == {k: int((ref == k).sum()) for k in (TILE_FULL, TILE_PARTIAL, TILE_EMPTY)}
+
+
+def test_training_sequence_tile_counts():
+    """The 144768-token training sequence (8 clean + 8 noisy chunks of 6032 tokens and an
+    8-chunk bidirectional block) has 1131 x 1131 tiles of 128: 300713 full, 2629 partial
+    and 975819 empty, counted from the row intervals and by the oracle's chunk-pair
+    reduction."""
+    expect = {TILE_FULL: 300713, TILE_PARTIAL: 2629, TILE_EMPTY: 975819}
+    assert sum(expect.values()) == 1131 * 1131
+    assert _tile_counts_by_intervals(8, 6032, 8) == expect
+    cls = classify_tiles_blocks(MobaLayout(8, 6032, 8), 128)
+    assert {k: int((cls == k).sum()) for k in expect} == expect
