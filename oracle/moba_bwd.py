@@ -100,6 +100,22 @@ def moba_dq_rows(q, k, v, do, lay: MobaLayout, rows: Iterable[int], scale: float
     return out
 
 
+def _rows_p_cols(q, k, v, do, rows, keys, cols, h, scale):
+    """P and dS of the given query rows (head h) on the key columns ``cols`` only.  The
+    row's normaliser and D = rowsum(dO o O) need the whole row over its readable
+    ``keys``; dS_ij = P_ij (dP_ij - D_i) is elementwise in j, so dP is formed on the
+    listed columns alone."""
+    z = scale * (q[rows, h] @ k[keys, h].T)
+    z = z - z.max(axis=1, keepdims=True)
+    e = np.exp(z)
+    p = e / e.sum(axis=1, keepdims=True)
+    o = p @ v[keys, h]
+    d = (do[rows, h] * o).sum(axis=1, keepdims=True)
+    p_c = p[:, cols]
+    dp_c = do[rows, h] @ v[keys[cols], h].T
+    return p_c, p_c * (dp_c - d)
+
+
 def moba_dkdv_keys(q, k, v, do, lay: MobaLayout, keys: Iterable[int], scale: float,
                    batch: int = 1024):
     """dK and dV of the listed key rows ([n, H, D] each): the sums over every query
@@ -118,7 +134,7 @@ def moba_dkdv_keys(q, k, v, do, lay: MobaLayout, keys: Iterable[int], scale: flo
         for b in range(0, sel.size, batch):
             r = readers[sel[b:b + batch]]
             for h in range(H):
-                p, ds = _rows_bwd(q, k, v, do, r, ks, h, scale)
-                dv[hit, h] += p[:, col[hit]].T @ do[r, h]
-                dk[hit, h] += scale * ds[:, col[hit]].T @ q[r, h]
+                p_c, ds_c = _rows_p_cols(q, k, v, do, r, ks, col[hit], h, scale)
+                dv[hit, h] += p_c.T @ do[r, h]
+                dk[hit, h] += scale * ds_c.T @ q[r, h]
     return dk, dv

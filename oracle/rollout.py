@@ -87,12 +87,15 @@ def rollout(spec, chunks, rows_for=None, use_rope: bool = True,
             pending_evicted = cache.evict(window_schedule[c])
             for f in pending_evicted:
                 store.pop(f, None)
+        rows = np.arange(q.shape[0]) if rows_for is None else np.asarray(rows_for(c, s))
         if use_rope:
+            # each token turns by the angles of its own position, so only the
+            # evaluated query rows need rotating
             t, hh, ww = rope_positions(frames, spec.grid_h, spec.grid_w)
-            q_rot = rope3d(q, t, hh, ww, pairs, spec.rope().base)
+            q_rot = rope3d(q[rows], t[rows], hh[rows], ww[rows], pairs, spec.rope().base)
             k_rot = rope3d(k, t, hh, ww, pairs, spec.rope().base)
         else:
-            q_rot, k_rot = q, k
+            q_rot, k_rot = q[rows], k
         vis = cache.cached_frames()
         k_aux, v_aux = [], []
         aux = aux_for(c) if aux_for is not None else None
@@ -105,8 +108,7 @@ def rollout(spec, chunks, rows_for=None, use_rope: bool = True,
             k_aux, v_aux = [ka], [va]
         k_all = np.concatenate([store[f][0] for f in vis] + k_aux + [k_rot], axis=0)
         v_all = np.concatenate([store[f][1] for f in vis] + v_aux + [v], axis=0)
-        rows = np.arange(q.shape[0]) if rows_for is None else np.asarray(rows_for(c, s))
-        o, lse = attention(q_rot[rows], k_all, v_all, scale)
+        o, lse = attention(q_rot, k_all, v_all, scale)
         res.outputs.append(o)
         res.lses.append(lse)
         res.rows.append(rows)

@@ -75,18 +75,33 @@ def test_multi_step_cache_read_unchanged():
     _compare_rollouts(spec, list(wl.rollout_chunks(spec)))
 
 
-def test_832x464_rollout_sampled_rows():
-    """Full 832x464 shapes (12 heads, d128, 1508 tokens/frame, 6 + 8 slots, 4-frame
-    chunks) over the fill-up chunks 0-4 and the first steady-state chunk."""
-    spec = wl.shrink(wl.VIDEO_832x464, n_chunks=6)
+def test_832x464_rollout_40_chunks():
+    """The whole 40-chunk 832x464 rollout (12 heads, d128, 1508 tokens/frame, 6 + 8 slots,
+    4-frame chunks; frames up to 159, the window wrapping ~19 times): every row of the
+    fill-up chunks 0-4 and of the last chunk 39; 1024 random rows plus the first 128 and
+    last 16 rows of every other chunk.  Slot maps after every append, bit-exact."""
+    spec = wl.VIDEO_832x464
     L = spec.chunk_tokens
+    every_row = {0, 1, 2, 3, 4, spec.n_chunks - 1}
 
     def rows_for(c, s):
-        always = list(range(128)) + list(range(L - 16, L)) + list(range(1408, 1664))
-        return wl.sample_rows(L, 256, 1000 + c, always)
+        if c in every_row:
+            return np.arange(L)
+        return wl.sample_rows(L, 1024, 1000 + c, list(range(128)) + list(range(L - 16, L)))
 
-    worst, got = _compare_rollouts(spec, list(wl.rollout_chunks(spec)), rows_for=rows_for)
-    print(f"832x464 worst max_abs={worst[0]:.3e} rel_rms={worst[1]:.3e}")
+    ref = rollout(spec, wl.rollout_chunks(spec), rows_for=rows_for)
+    got = gpu_rollout(spec, wl.rollout_chunks(spec), rows_for=rows_for)
+    assert len(got["outputs"]) == spec.n_chunks
+    worst = (0.0, 0.0)
+    for n, (o, o_ref, l, l_ref) in enumerate(zip(got["outputs"], ref.outputs, got["lses"],
+                                                 ref.lses)):
+        ma, rr = assert_close(o, o_ref, f"chunk {n}")
+        assert np.abs(l - l_ref).max() <= TOL_LSE, f"chunk {n}: lse"
+        worst = (max(worst[0], ma), max(worst[1], rr))
+    assert got["slot_maps"] == ref.slot_maps
+    assert [a[0] for a in got["appended"]] == ref.appended_slots
+    assert ref.n_keys[-1] == 27144
+    print(f"832x464 40-chunk rollout: worst max_abs={worst[0]:.3e} rel_rms={worst[1]:.3e}")
 
 
 def test_append_writes_rotated_k_and_exact_v():

@@ -164,6 +164,31 @@ def test_full_size_sampled():
          assert_grad_close(got_dv, ref_dv, "dv full")]
     print("moba bwd full-size (max_abs/max|ref|, rel_rms) dq/dk/dv:", r)
 
+    # key blocks read by many query chunks, element-wise on a few heads (the oracle
+    # evaluates every reader's whole row of P): C1 (read by all 8 clean chunks and noisy
+    # chunks 2-8), C8, N8 and both ends of the bidirectional block (read by all of B)
+    def keyset(start, n_edge, n_rand, seed):
+        ks = set(range(start, start + n_edge)) | set(range(start + c - n_edge, start + c))
+        ks |= set((wl.sample_rows(c, n_rand, seed) + start).tolist())
+        return np.array(sorted(ks))
+    heavy = [("C1", keyset(0, 8, 16, 1012), [0, 6]),
+             ("C8", keyset(7 * c, 8, 16, 1013), [3, 11]),
+             ("N8", keyset(nc + 7 * c, 8, 16, 1014), [5, 8]),
+             ("B ends", np.array(list(range(2 * nc, 2 * nc + 16)) + list(range(L - 16, L))),
+              [1, 7])]
+    for name, keys, heads in heavy:
+        kidx = torch.from_numpy(keys).cuda()
+        got_k = to_np(dk.index_select(0, kidx))[:, heads]
+        got_v = to_np(dv.index_select(0, kidx))[:, heads]
+        ref_k, ref_v = np.zeros_like(got_k), np.zeros_like(got_v)
+        for j, h in enumerate(heads):
+            sl = slice(h, h + 1)
+            ref_k[:, j:j + 1], ref_v[:, j:j + 1] = mb.moba_dkdv_keys(
+                q[:, sl], k[:, sl], v[:, sl], do[:, sl], lay, keys, scale)
+        rk = assert_grad_close(got_k, ref_k, f"dk {name}")
+        rv = assert_grad_close(got_v, ref_v, f"dv {name}")
+        print(f"moba bwd full-size dk/dv on {name} keys, heads {heads}: {rk} {rv}")
+
     sum_dk = dk.float().sum(0).double().cpu().numpy()               # [H, D]
     sum_dv = dv.float().sum(0).double().cpu().numpy()
     sum_do = do.astype(np.float64).sum(0)

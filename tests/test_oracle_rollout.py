@@ -114,3 +114,20 @@ def test_cross_attention_reads_env_and_own_prompt_only():
         ob, _ = masked_attention(q, allk, allv, allowed, 0.3)
         o, _ = attention(q, np.concatenate([env_k, loc[t][0]]), np.concatenate([env_v, loc[t][1]]), 0.3)
         np.testing.assert_allclose(o, ob, atol=1e-13)
+
+
+def test_checked_rows_equal_the_full_rollout_rows():
+    """Evaluating a subset of query rows gives those rows of the full rollout, up to the
+    order of fp64 rounding inside the library matmul (RoPE turns each token by its own
+    position; attention is row by row)."""
+    spec = wl.shrink(wl.VIDEO_832x464, grid_h=3, grid_w=5, heads=2, head_dim=64, chunk_frames=2,
+                     sinks=1, window=2, n_chunks=4, seed=41)
+    items = list(wl.rollout_chunks(spec))
+    full = rollout(spec, items)
+    pick = {c: np.array(sorted({0, 7, 29, c + 3})) for c in range(spec.n_chunks)}
+    part = rollout(spec, items, rows_for=lambda c, s: pick[c])
+    for n, it in enumerate(items):
+        rows = pick[it["chunk"]]
+        np.testing.assert_allclose(part.outputs[n], full.outputs[n][rows], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(part.lses[n], full.lses[n][:, rows], rtol=0, atol=1e-13)
+    assert part.slot_maps == full.slot_maps
