@@ -597,6 +597,9 @@ def run_moba(args) -> dict:
     from kv_cache_chunk_ring_b200 import kvcr
     _build.build()
     spec = wl.MOBA_8x6032
+    if args.moba_chunk_tokens:                        # a smaller sequence of the same shape
+        spec = dataclasses.replace(spec, name=f"moba_8chunks_x{args.moba_chunk_tokens}",
+                                   chunk_tokens=args.moba_chunk_tokens)
     gen = torch.Generator(device="cuda").manual_seed(spec.seed)
     shape = (spec.seq_len, spec.heads, spec.head_dim)
     q, k, v = (_randn(shape, gen) for _ in range(3))
@@ -790,6 +793,70 @@ def run_aux(args) -> dict:
             "steps": args.steps, "warmup": args.warmup}
 
 
+def fp8_mixed_peak(bf16_peak: float) -> float:
+    """Peak of the e4m3-QK^T attention's tensor work: half of the useful FLOPs (Q K^T)
+    run at the e4m3 rate, nominally twice the bf16 rate, the other half (P V) at the
+    bf16 rate, so 4 / (2 / 2 + 2 / 1) = 4/3 of the bf16 peak."""
+    return bf16_peak * 4.0 / 3.0
+
+
+def run_fp8(args) -> dict:
+    """832x464 steady-state chunk step with the QK^T product in e4m3: stage (RoPE of Q
+    and the chunk's K), e4m3 quantization of both, attention over 6 + 8 cached + 4
+    current frames (27144 keys) reading the cache's e4m3 K copies, append (bf16 K/V
+    and their e4m3 K copy)."""
+    import torch
+    from kv_cache_chunk_ring_b200 import build as _build
+    from kv_cache_chunk_ring_b200 import kvcr
+    _build.build()
+    spec = SPEC
+    T, H, D, F = spec.tokens_per_frame, spec.heads, spec.head_dim, spec.chunk_frames
+    cache = kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope(), fp8_k=True)
+    gen = torch.Generator(device="cuda").manual_seed(spec.seed)
+    pool = [tuple(_randn((spec.chunk_tokens, H, D), gen) for _ in range(3)) for _ in range(3)]
+    o = torch.empty_like(pool[0][0])
+    state = {"c": 0}
+
+    def step():
+        c = state["c"]
+        frames = list(range(c * F, (c + 1) * F))
+        q, k, v = pool[c % 3]
+        cache.attention(q, k, v, frames, out=o, fp8=True)
+        cache.append(k, v, frames)
+        state["c"] = c + 1
+
+    for _ in range(STEADY_CHUNK):
+        step()
+    ms = _timed(step, args.steps, args.warmup)
+    kvcr.kvcr_trace_reset()
+    kvcr.kvcr_trace_enable(True)
+    for _ in range(max(3, min(args.steps, 20))):
+        step()
+    torch.cuda.synchronize()
+    kvcr.kvcr_trace_enable(False)
+    kt = {name: kvcr.kvcr_trace_read(kid) for kid, name in kvcr.KERNEL_NAMES.items()}
+    kvcr.kvcr_trace_reset()
+    kvcr.kvcr_check_status()
+    peaks, kind = load_peaks()
+    flops = step_flops(spec)
+
+    def avg(name):
+        n, t = kt[name]
+        return t / max(1, n)
+    attn_ms = avg("chunk_attn_fp8")
+    tf = flops / (attn_ms * 1e-3) / 1e12
+    peak = fp8_mixed_peak(float(peaks["bf16_tflops"]))
+    return {"workload": spec.name + "_qk_e4m3", "ms_per_step": round(ms, 4),
+            "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": UNIT,
+            "dtype": "e4m3 QK^T, bf16 P V, fp32 accumulate",
+            "attn_kernel_ms": round(attn_ms, 4), "attn_tflops": round(tf, 1),
+            "attn_frac_of_mixed_peak": round(tf / peak, 4), "mixed_peak_tflops": round(peak, 1),
+            "attn_frac_of_bf16_peak": round(tf / float(peaks["bf16_tflops"]), 4),
+            "peak_source": f"{kind} bf16_tflops x 4/3 (Q K^T at the nominal e4m3 rate, 2x bf16)",
+            "kernels_ms": {k: round(avg(k), 5) for k, (n, _) in kt.items() if n},
+            "steps": args.steps, "warmup": args.warmup}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -803,9 +870,10 @@ def main():
                     help="multi-GPU partition: heads of one layer cache per rank (strong "
                          "scaling) or one layer cache per rank (weak scaling)")
     ap.add_argument("--moba-chunk-tokens", type=int, default=0,
-                    help="moba_bwd: tokens per chunk (default: the workload's 6032); a smaller "
+                    help="moba, moba_bwd: tokens per chunk (default: the workload's 6032); a smaller "
                          "value gives a case small enough for a full profiler capture")
-    ap.add_argument("--workload", default="chunk", choices=["chunk", "layers30", "moba", "moba_bwd", "dynwin", "aux"],
+    ap.add_argument("--workload", default="chunk",
+                    choices=["chunk", "layers30", "moba", "moba_bwd", "dynwin", "aux", "fp8"],
                     help="chunk: the 832x464 steady-state step (the bench line); the others "
                          "print single-GPU timings of the other workloads")
     args = ap.parse_args()
@@ -828,7 +896,7 @@ def main():
         return
     if args.workload != "chunk":
         fn = {"layers30": run_layers30, "moba": run_moba, "moba_bwd": run_moba_bwd,
-              "dynwin": run_dynwin, "aux": run_aux}[args.workload]
+              "dynwin": run_dynwin, "aux": run_aux, "fp8": run_fp8}[args.workload]
         if rank == 0:
             print(json.dumps(fn(args)))
         return

@@ -155,6 +155,29 @@ int kv_cache_init_aux(kvcr_cache **out, int sinks, int window, int aux_frames,
 int kv_cache_set_aux(kvcr_cache *c, const void *k, const void *v, const int32_t *aux_pos,
                      int n_frames, void *stream);
 
+/* Cache flags of kv_cache_init_ex(). */
+enum {
+    /* Keep, beside the bf16 K of every cached and auxiliary frame, an e4m3 copy of
+     * it with one fp32 scale per block of 128 tokens and head, written by the same
+     * append / set_aux call; chunk_attention_fwd_fp8() reads it.  Needs bf16 and
+     * head_dim 128. */
+    KVCR_CACHE_FP8_K = 1
+};
+
+/* kv_cache_storage_bytes_aux() / kv_cache_init_aux() with cache flags (0 or
+ * KVCR_CACHE_FP8_K).  With KVCR_CACHE_FP8_K the storage also holds the e4m3 K
+ * copies (T * H * D bytes per frame slot), their scales (4 * ceil(T / 128) * H
+ * bytes per slot) and the e4m3 staging of one chunk's queries and keys.
+ * kv_cache_init_ex returns KVCR_EUNSUPPORTED for KVCR_CACHE_FP8_K with fp32 or
+ * head_dim 64, KVCR_EINVAL for unknown flags. */
+size_t kv_cache_storage_bytes_ex(int sinks, int window, int aux_frames, int tokens_per_frame,
+                                 int heads, int head_dim, int chunk_frames, int with_rope,
+                                 kvcr_dtype dtype, unsigned flags);
+int kv_cache_init_ex(kvcr_cache **out, int sinks, int window, int aux_frames,
+                     int tokens_per_frame, int heads, int head_dim, int chunk_frames,
+                     const kvcr_rope *rope, kvcr_dtype dtype, unsigned flags,
+                     void *device_storage, size_t storage_bytes);
+
 /* Number of auxiliary frames the next attention call reads (0 after the chunk's
  * append; see kv_cache_set_aux).  Host only; KVCR_EINVAL for NULL arguments. */
 int kv_cache_num_aux(const kvcr_cache *c, int *n);
@@ -215,6 +238,14 @@ int kv_cache_last_append(const kvcr_cache *c, int32_t *slots, int slots_cap,
 /* Number of cached frames (library convention; host only). */
 int kv_cache_num_cached(const kvcr_cache *c, int *n);
 
+/* Device addresses of the e4m3 copy of slot `slot`'s K: codes [tokens_per_frame]
+ * [heads][head_dim] (one byte each; the block of tokens 128 b .. 128 b + 127 and
+ * head h dequantizes to code * scales[b * heads + h]) and scales fp32
+ * [ceil(tokens_per_frame / 128)][heads].  Only for caches made with
+ * KVCR_CACHE_FP8_K (else KVCR_ESTATE).  For reading back or checking the copy. */
+int kv_cache_slot_data_fp8(const kvcr_cache *c, int slot, const void **k_codes,
+                           const float **k_scales);
+
 /* Device addresses of slot `slot`'s K and V, each [tokens_per_frame][heads][head_dim]
  * in the cache dtype (K stored rotated).  For reading back or saving a cache.
  * Slots sinks + window .. + aux_frames - 1 are the auxiliary slots. */
@@ -265,6 +296,25 @@ int chunk_attention_fwd_static_scratch(kvcr_cache *c, const void *q, int n_q,
                                        const void *k_cur, const void *v_cur,
                                        const int32_t *cur_frame_idx, int n_cur_frames,
                                        float softmax_scale, void *o, float *lse, void *stream);
+
+/* chunk_attention_fwd() with the QK^T product in 8 bits: the pages' own speed
+ * lever on this path is an 8-bit QK^T (kaarelkaarelson.com/lingbot, kernel table,
+ * "SageAttention" row: INT8 QK^T at 65 % of the RTX 5090's INT8 peak); here it is
+ * the tensor cores' e4m3 (tcgen05.mma kind::f8f6f4), with P V in bf16.  The
+ * rotated queries and current keys (bf16, as chunk_attention_fwd() stages them)
+ * and every cached or auxiliary K are block-quantized: per block of 128 tokens
+ * and head, amax = max |x|, scale = amax / 448, code = e4m3(x * (448 / amax))
+ * rounded to nearest even and saturated (fp32 arithmetic); blocks are 128 tokens
+ * of one cached / auxiliary frame, and 128 tokens of the chunk for its own Q and
+ * K.  The scores are (Q codes . K codes) * q scale * k scale * softmax_scale;
+ * everything after them is as in chunk_attention_fwd() (fp32 softmax, bf16 P,
+ * fp32 accumulation of P V).  Arguments, outputs and errors are those of
+ * chunk_attention_fwd(); additionally KVCR_ESTATE when the cache was made without
+ * KVCR_CACHE_FP8_K, and KVCR_ESHAPE when a cache without RoPE gets n_q >
+ * chunk_frames * tokens_per_frame (the size of the query staging). */
+int chunk_attention_fwd_fp8(kvcr_cache *c, const void *q, int n_q, const void *k_cur,
+                            const void *v_cur, const int32_t *cur_frame_idx, int n_cur_frames,
+                            float softmax_scale, void *o, float *lse, void *stream);
 
 /* Attention under the MoBA mask over one sequence of L = layout tokens ("Infinite
  * Worlds with Versatile Interactions", causal-pretraining paragraph: the
@@ -351,7 +401,9 @@ enum {
     KVCR_K_MOBA_BWD_DQ = 7,   /* MoBA backward: dQ (tensor cores) */
     KVCR_K_SET_AUX = 8,       /* auxiliary frames written into their slots (RoPE3D of K) */
     KVCR_K_APPEND_BATCH = 9,  /* one cache write for several caches (RoPE3D of K) */
-    KVCR_K_COUNT = 10
+    KVCR_K_QUANT_E4M3 = 10,   /* e4m3 block quantization of K (cache) or Q / current K */
+    KVCR_K_CHUNK_ATTN_FP8 = 11, /* tensor-core chunk attention, e4m3 QK^T, bf16 P V */
+    KVCR_K_COUNT = 12
 };
 
 /* Count of every kernel the library launched in this process (library

@@ -86,14 +86,20 @@ struct __align__(8) Ctl {
   uint16_t tiles[kMobaMaxTiles];  // MoBA: key tile | class(tile 0) << 12 | class(tile 1) << 14
 };
 
-template <int HD>
+// kFp8: Q and K tiles hold e4m3 codes (one 128-byte box per 128-element row);
+// V stays bf16.
+template <int HD, bool kFp8>
 struct Smem {
-  static constexpr int kBoxes = HD / 64;          // 64-element (128-byte) boxes per row
+  static_assert(!kFp8 || HD == 128, "e4m3 QK^T tiles need head_dim 128");
+  static constexpr int kBoxes = HD / 64;          // 64-element (128-byte) bf16 boxes per row
   static constexpr int kBoxBytes = 128 * 128;     // 128 rows x 128 bytes
-  static constexpr int kTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;                   // V tile
+  static constexpr int kQKBoxes = kFp8 ? HD / 128 : kBoxes;              // Q / K boxes per row
+  static constexpr int kQKBoxElems = kFp8 ? 128 : 64;
+  static constexpr int kQKTileBytes = kQKBoxes * kBoxBytes;               // Q / K tile
   static constexpr int kQ = 0;                    // Q0, Q1
-  static constexpr int kK = kQ + 2 * kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kK = kQ + 2 * kQKTileBytes;
+  static constexpr int kV = kK + kStages * kQKTileBytes;
   static constexpr int kCtl = kV + kStages * kTileBytes;
   static constexpr int kBytes = kCtl + (int)sizeof(Ctl) + 1024;  // + 1024 B alignment slack
 };
@@ -181,25 +187,30 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int HD>
+template <int HD, bool kFp8>
 __device__ __forceinline__ void load_kv_tile(const ChunkAttnParams& p, const TileRef& t, bool is_v,
                                              uint8_t* dst, uint64_t* bar, int h) {
+  using L = Smem<HD, kFp8>;
+  const int n_box = is_v ? L::kBoxes : L::kQKBoxes;
+  const int box_elems = is_v ? 64 : L::kQKBoxElems;
 #pragma unroll
-  for (int b = 0; b < Smem<HD>::kBoxes; ++b) {
-    uint8_t* d = dst + b * Smem<HD>::kBoxBytes;
+  for (int b = 0; b < L::kBoxes; ++b) {
+    if (b >= n_box) break;
+    uint8_t* d = dst + b * L::kBoxBytes;
     if (t.map == 0)
-      tma_load_4d(d, is_v ? &p.tm_vc : &p.tm_kc, bar, b * 64, h, t.row0, t.slot);
+      tma_load_4d(d, is_v ? &p.tm_vc : &p.tm_kc, bar, b * box_elems, h, t.row0, t.slot);
     else
-      tma_load_3d(d, is_v ? &p.tm_vn : &p.tm_kn, bar, b * 64, h, t.row0);
+      tma_load_3d(d, is_v ? &p.tm_vn : &p.tm_kn, bar, b * box_elems, h, t.row0);
   }
 }
 
-template <int HD>
+template <int HD, bool kFp8>
 __device__ __forceinline__ void load_kv_tile(const MobaAttnParams& p, const TileRef& t, bool is_v,
                                              uint8_t* dst, uint64_t* bar, int h) {
 #pragma unroll
-  for (int b = 0; b < Smem<HD>::kBoxes; ++b)
-    tma_load_3d(dst + b * Smem<HD>::kBoxBytes, is_v ? &p.tm_v : &p.tm_k, bar, b * 64, h, t.row0);
+  for (int b = 0; b < Smem<HD, false>::kBoxes; ++b)
+    tma_load_3d(dst + b * Smem<HD, false>::kBoxBytes, is_v ? &p.tm_v : &p.tm_k, bar, b * 64, h,
+                t.row0);
 }
 
 __device__ __forceinline__ void prefetch_maps(const ChunkAttnParams& p) {
@@ -252,6 +263,13 @@ __device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
   return upto_hi & ~((1u << lo) - 1u);
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 2^x on the SFU (MUFU.EX2); -inf -> +0.
 __device__ __forceinline__ float ex2_sfu(float x) {
   float y;
@@ -289,9 +307,24 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int HD, bool kMoba, typename Params>
+// Scale of the e4m3 key block of tile t for head h (chunk attention).
+__device__ __forceinline__ float key_block_scale(const ChunkAttnParams& p, const TileRef& t, int h) {
+  const int blk = t.row0 >> 7;
+  return t.map == 0 ? __ldg(p.kc_scale + ((size_t)t.slot * p.s.tiles_per_slot + blk) * p.c.H + h)
+                    : __ldg(p.kn_scale + (size_t)blk * p.c.H + h);
+}
+__device__ __forceinline__ float key_block_scale(const MobaAttnParams&, const TileRef&, int) {
+  return 1.f;
+}
+__device__ __forceinline__ float query_block_scale(const ChunkAttnParams& p, int q_tile, int h) {
+  return q_tile * kTile < p.c.n_q ? __ldg(p.q_scale + (size_t)q_tile * p.c.H + h) : 0.f;
+}
+__device__ __forceinline__ float query_block_scale(const MobaAttnParams&, int, int) { return 1.f; }
+
+template <int HD, bool kMoba, bool kFp8, typename Params>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ Params p) {
-  using L = Smem<HD>;
+  static_assert(!(kMoba && kFp8), "the MoBA kernel is bf16 only");
+  using L = Smem<HD, kFp8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + L::kCtl);
@@ -347,13 +380,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     // ------------------------------------------------------ TMA producer --
     if (lane == 0 && n_tiles > 0) {
       prefetch_maps(p);
-      mbar_arrive_expect_tx(&ctl->q_full, 2 * L::kTileBytes);
+      mbar_arrive_expect_tx(&ctl->q_full, 2 * L::kQKTileBytes);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int b = 0; b < L::kBoxes; ++b)
-          tma_load_3d(smem + L::kQ + t * L::kTileBytes + b * L::kBoxBytes, &p.tm_q, &ctl->q_full,
-                      b * 64, h, q0 + t * kTile);
+        for (int b = 0; b < L::kQKBoxes; ++b)
+          tma_load_3d(smem + L::kQ + t * L::kQKTileBytes + b * L::kBoxBytes, &p.tm_q,
+                      &ctl->q_full, b * L::kQKBoxElems, h, q0 + t * kTile);
       int issued = 0;  // tiles whose K and V loads were issued
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
@@ -361,15 +394,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const uint32_t ph = (uint32_t)(j / kStages) & 1u;
         const TileRef t = tile_ref(p, ctl, j);
         if (!(ok = wait_bar(&ctl->k_empty[st], ph ^ 1u, ctl))) break;
-        mbar_arrive_expect_tx(&ctl->k_full[st], L::kTileBytes);
-        load_kv_tile<HD>(p, t, false, smem + L::kK + st * L::kTileBytes, &ctl->k_full[st], h);
+        mbar_arrive_expect_tx(&ctl->k_full[st], L::kQKTileBytes);
+        load_kv_tile<HD, kFp8>(p, t, false, smem + L::kK + st * L::kQKTileBytes, &ctl->k_full[st],
+                               h);
         if (!(ok = wait_bar(&ctl->v_empty[st], ph ^ 1u, ctl))) {
           issued = j;
           drain_wait(&ctl->k_full[st], ph);
           break;
         }
         mbar_arrive_expect_tx(&ctl->v_full[st], L::kTileBytes);
-        load_kv_tile<HD>(p, t, true, smem + L::kV + st * L::kTileBytes, &ctl->v_full[st], h);
+        load_kv_tile<HD, kFp8>(p, t, true, smem + L::kV + st * L::kTileBytes, &ctl->v_full[st], h);
         issued = j + 1;
       }
       if (!ok) {
@@ -386,21 +420,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   } else if (warp == kWarpMma) {
     // -------------------------------------------------------- MMA issuer --
     if (lane == 0 && n_tiles > 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t kIdescS =
+          kFp8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, false);
       constexpr uint32_t kIdescO = idesc_bf16_f32(128, HD, true);
       const uint32_t sQ = smem_u32(smem + L::kQ);
       const uint32_t sK = smem_u32(smem + L::kK);
       const uint32_t sV = smem_u32(smem + L::kV);
-      // S_t(j) = Q_t K_j^T
+      // S_t(j) = Q_t K_j^T: K steps of 32 bytes (16 bf16 or 32 e4m3 elements) inside
+      // each 128-byte swizzled row
       auto issue_s = [&](int t, int j) {
         const uint32_t d = tmem + kTmemS + (uint32_t)t * 128u;
-        const uint32_t qb = sQ + t * L::kTileBytes;
-        const uint32_t kb = sK + (j % kStages) * L::kTileBytes;
+        const uint32_t qb = sQ + t * L::kQKTileBytes;
+        const uint32_t kb = sK + (j % kStages) * L::kQKTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
+        for (int kk = 0; kk < HD / (kFp8 ? 32 : 16); ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          umma_ss(d, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescS,
-                  kk > 0 ? 1u : 0u);
+          if constexpr (kFp8)
+            umma_ss_f8(d, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                       kIdescS, kk > 0 ? 1u : 0u);
+          else
+            umma_ss(d, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescS,
+                    kk > 0 ? 1u : 0u);
         }
       };
       // O_t += P_t(j) V_j over part hf of the keys, P_t in TMEM (8 packed columns
@@ -477,6 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t s_addr = tmem + lane_base + kTmemS + (uint32_t)tq * 128u;
     const uint32_t o_addr = tmem + lane_base + kTmemO + (uint32_t)tq * 128u;
     const float sl2 = p.c.scale_log2;
+    // e4m3 QK^T: S holds code products; a tile's true scores are S * (q scale * k scale)
+    const float q_blk_scale = kFp8 ? query_block_scale(p, 2 * unit + tq, h) : 1.f;
     const int row_g = q0 + tq * kTile + r;           // global query row
     float m_ref = -INFINITY;                        // running (possibly stale) max, log2 units
     float l_sum = 0.f;
@@ -494,6 +536,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
     for (int j = 0; j < n_tiles; ++j) {
       const TileRef t = tile_ref(p, ctl, j);        // independent of S: before the wait
+      float sl2t = sl2;                              // log2-domain factor of this tile's S
+      if constexpr (kFp8) {
+        // a zero block scale gives zero scores: keep the factor positive so that the
+        // masked -inf entries stay -inf
+        sl2t = fmaxf(sl2 * q_blk_scale * key_block_scale(p, t, h), 1.17549435e-38f);
+      }
       ok = wait_bar(&ctl->s_full[tq], (uint32_t)j & 1u, ctl);
       if (!__all_sync(0xFFFFFFFFu, ok)) {  // leave the loop warp-uniformly
         ok = false;
@@ -520,18 +568,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             if (!((keep >> n) & 1u)) s[32 * c + n] = __float_as_uint(-INFINITY);
         }
       }
-      float mx[16];                                 // 16 independent chains, then a tree
+      // row max with three-input max: 16 independent chains, then a tree (72 max
+      // instructions for 128 keys)
+      float mx[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) mx[k] = __uint_as_float(s[k]);
+      for (int k = 0; k < 16; ++k)
+        mx[k] = fmax3(__uint_as_float(s[k]), __uint_as_float(s[16 + k]),
+                      __uint_as_float(s[32 + k]));
 #pragma unroll
-      for (int n = 16; n < 128; n += 16)
+      for (int n = 48; n < 112; n += 32)
 #pragma unroll
-        for (int k = 0; k < 16; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(s[n + k]));
+        for (int k = 0; k < 16; ++k)
+          mx[k] = fmax3(mx[k], __uint_as_float(s[n + k]), __uint_as_float(s[n + 16 + k]));
 #pragma unroll
-      for (int w = 8; w >= 1; w >>= 1)
+      for (int k = 0; k < 16; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(s[112 + k]));
+      float mt[6];
 #pragma unroll
-        for (int k = 0; k < w; ++k) mx[k] = fmaxf(mx[k], mx[k + w]);
-      const float m_new = fmaxf(m_ref, mx[0] * sl2);
+      for (int k = 0; k < 5; ++k) mt[k] = fmax3(mx[3 * k], mx[3 * k + 1], mx[3 * k + 2]);
+      mt[5] = mx[15];
+      const float row_max = fmaxf(fmax3(mt[0], mt[1], mt[2]), fmax3(mt[3], mt[4], mt[5]));
+      const float m_new = fmaxf(m_ref, row_max * sl2t);
 
       // O_t is stable here: S_t(j) was committed after PV_t(j-1).
       const bool grow = m_new > m_ref + kRescaleLog2;
@@ -552,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (m_new != -INFINITY) m_ref = m_new;
       }
       const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
-      const float2 sl2x2 = make_float2(sl2, sl2);
+      const float2 sl2x2 = make_float2(sl2t, sl2t);
       const float2 negm = make_float2(-msub, -msub);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {                 // 4 groups of 32 keys -> 16 packed columns
@@ -640,38 +696,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   }
 }
 
-template <int HD, bool kMoba, typename Params>
+template <int HD, bool kMoba, bool kFp8, typename Params>
 cudaError_t launch_impl(const Params& p, dim3 grid, cudaStream_t s) {
-  auto kern = attn_fwd_kernel<HD, kMoba, Params>;
+  auto kern = attn_fwd_kernel<HD, kMoba, kFp8, Params>;
   // the shared-memory limit is a per-device attribute of the function
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<HD>::kBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Smem<HD, kFp8>::kBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  kern<<<grid, kThreads, Smem<HD>::kBytes, s>>>(p);
+  kern<<<grid, kThreads, Smem<HD, kFp8>::kBytes, s>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_chunk_attn_sm100(const ChunkAttnParams& p, int head_dim, int n_q_tiles,
-                                    cudaStream_t s) {
+                                    cudaStream_t s, bool qk_e4m3) {
   dim3 grid((unsigned)((n_q_tiles + 1) / 2), (unsigned)p.c.H);
-  if (head_dim == 128) return launch_impl<128, false>(p, grid, s);
-  if (head_dim == 64) return launch_impl<64, false>(p, grid, s);
+  if (qk_e4m3) {
+    if (head_dim == 128) return launch_impl<128, false, true>(p, grid, s);
+    return cudaErrorInvalidValue;
+  }
+  if (head_dim == 128) return launch_impl<128, false, false>(p, grid, s);
+  if (head_dim == 64) return launch_impl<64, false, false>(p, grid, s);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_moba_attn_sm100(const MobaAttnParams& p, int head_dim, cudaStream_t s) {
   dim3 grid((unsigned)(p.s.n_row_tiles * p.c.H));
-  if (head_dim == 128) return launch_impl<128, true>(p, grid, s);
-  if (head_dim == 64) return launch_impl<64, true>(p, grid, s);
+  if (head_dim == 128) return launch_impl<128, true, false>(p, grid, s);
+  if (head_dim == 64) return launch_impl<64, true, false>(p, grid, s);
   return cudaErrorInvalidValue;
 }
 

@@ -24,6 +24,7 @@
 #include <cstdio>
 #include <cstring>
 #include <deque>
+#include <memory>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -69,29 +70,35 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tiled map over a bf16 tensor [..][tokens][H][D] (innermost first: D, H,
-// tokens[, slots]); box = 64 x 1 x box_rows (x 1), 128-byte swizzle, zero fill.
-int encode_bf16_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                    int box_rows) {
+// Tiled map over a tensor [..][tokens][H][D] of bf16 (box 64 elements wide) or
+// of e4m3 codes as bytes (box 128 wide), innermost first: D, H, tokens[,
+// slots]; box = 128 bytes x 1 x box_rows (x 1), 128-byte swizzle, zero fill.
+int encode_map(CUtensorMap* m, bool codes, const void* base, int rank, const uint64_t* dims,
+               int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(KVCR_ECUDA, "cuTensorMapEncodeTiled not available from the driver");
   cuuint64_t gdim[4];
   cuuint64_t gstride[3];
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t box[4] = {codes ? 128u : 64u, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  uint64_t stride = 2;
+  uint64_t stride = codes ? 1 : 2;
   for (int i = 0; i < rank; ++i) {
     gdim[i] = dims[i];
     if (i > 0) gstride[i - 1] = stride;
     stride *= dims[i];
   }
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
-                  gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, codes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  (cuuint32_t)rank, const_cast<void*>(base), gdim, gstride, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KVCR_ECUDA, "cuTensorMapEncodeTiled failed (" +
                                                      std::to_string((int)r) + ")");
   return KVCR_OK;
+}
+
+int encode_bf16_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                    int box_rows) {
+  return encode_map(m, false, base, rank, dims, box_rows);
 }
 
 // --------------------------------------------------------- failure hook --
@@ -162,11 +169,17 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct StorageLayout {
-  size_t k_off, v_off, q_off, ks_off, h_off, w_off, total;
+  size_t k_off, v_off, q_off, ks_off, h_off, w_off;
+  // e4m3 copies (KVCR_CACHE_FP8_K): cached K codes and their block scales, then the
+  // codes and scales of one chunk's queries and current keys
+  size_t k8_off, k8s_off, q8_off, q8s_off, c8_off, c8s_off;
+  size_t total;
 };
 
+int blocks_of(long long n) { return (int)((n + 127) / 128); }
+
 bool make_layout(int S, int W, int A, int T, int H, int D, int F, bool rope, size_t esize,
-                 StorageLayout* L) {
+                 StorageLayout* L, bool fp8 = false) {
   if (S < 0 || W < 0 || A < 0 || S + W < 1 || S + W + A > kMaxSlots || T < 1 || H < 1 || D < 1 ||
       F < 1 || F > kMaxFrames)
     return false;
@@ -189,6 +202,23 @@ bool make_layout(int S, int W, int A, int T, int H, int D, int F, bool rope, siz
     L->w_off = off;
     off = align_up(off + (size_t)T * (D / 2) * sizeof(float2), 256);
   }
+  L->k8_off = L->k8s_off = L->q8_off = L->q8s_off = L->c8_off = L->c8s_off = off;
+  if (fp8) {
+    const size_t codes = (size_t)T * H * D;                      // bytes per frame
+    const size_t chunk_codes = (size_t)F * T * H * D;
+    L->k8_off = off;
+    off = align_up(off + slots * codes, 256);
+    L->k8s_off = off;
+    off = align_up(off + slots * blocks_of(T) * H * sizeof(float), 256);
+    L->q8_off = off;
+    off = align_up(off + chunk_codes, 256);
+    L->q8s_off = off;
+    off = align_up(off + (size_t)blocks_of((long long)F * T) * H * sizeof(float), 256);
+    L->c8_off = off;
+    off = align_up(off + chunk_codes, 256);
+    L->c8s_off = off;
+    off = align_up(off + (size_t)blocks_of((long long)F * T) * H * sizeof(float), 256);
+  }
   L->total = off;
   return true;
 }
@@ -209,6 +239,8 @@ struct kvcr_cache {
   StorageLayout lay;
   int n_sm, cc_major;
   CUtensorMap tm_kc, tm_vc;
+  bool fp8;             // e4m3 K copies kept (KVCR_CACHE_FP8_K)
+  CUtensorMap tm_kc8;   // 4D map over the e4m3 K copies
   // slot table
   std::vector<int> slot_frame;
   int n_sinks_filled;
@@ -291,6 +323,32 @@ void fill_common(const kvcr_cache* c, RopeCopyParams& p) {
   p.wtab = c->rope ? reinterpret_cast<const float2*>(c->storage + c->lay.w_off) : nullptr;
 }
 
+// Segment i of a quantization launch: the bf16 K of physical slot `slot` of cache c
+// to its e4m3 copy and block scales.
+void quant_segment_of_slot(const kvcr_cache* c, int slot, QuantParams& p, int i, int tile0) {
+  const size_t codes = (size_t)c->T * c->H * c->D;
+  p.src[i] = c->storage + c->lay.k_off + (size_t)slot * codes * c->esize;
+  p.dst[i] = c->storage + c->lay.k8_off + (size_t)slot * codes;
+  p.scale[i] = reinterpret_cast<float*>(c->storage + c->lay.k8s_off) +
+               (size_t)slot * blocks_of(c->T) * c->H;
+  p.n_tok[i] = c->T;
+  p.tile0[i] = tile0;
+}
+
+// e4m3 copies of the K of the listed physical slots of an e4m3 cache (their bf16 K
+// written earlier on the same stream).
+cudaError_t quant_slots(const kvcr_cache* c, const std::vector<int>& slots, cudaStream_t s) {
+  if (!c->fp8 || slots.empty()) return cudaSuccess;
+  std::unique_ptr<QuantParams> p(new QuantParams());
+  std::memset(p.get(), 0, sizeof(QuantParams));
+  for (size_t i = 0; i < slots.size(); ++i)
+    quant_segment_of_slot(c, slots[i], *p, (int)i, (int)i * blocks_of(c->T));
+  p->n_seg = (int)slots.size();
+  p->H = c->H;
+  LaunchScope scope(KVCR_K_QUANT_E4M3, s);
+  return launch_quant_e4m3(*p, c->D, s);
+}
+
 int check_frames(const kvcr_cache* c, const int32_t* frames, int n, const char* what) {
   if (n > 0 && frames == nullptr) return fail(KVCR_EINVAL, std::string(what) + ": frame indices are NULL");
   int prev = c->last_frame;
@@ -310,15 +368,24 @@ extern "C" {
 
 const char* kvcr_last_error(void) { return g_err.c_str(); }
 
+size_t kv_cache_storage_bytes_ex(int sinks, int window, int aux_frames, int tokens_per_frame,
+                                 int heads, int head_dim, int chunk_frames, int with_rope,
+                                 kvcr_dtype dtype, unsigned flags) {
+  if (dtype != KVCR_BF16 && dtype != KVCR_F32) return 0;
+  if (flags & ~(unsigned)KVCR_CACHE_FP8_K) return 0;
+  StorageLayout L;
+  if (!make_layout(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
+                   with_rope != 0, dtype == KVCR_BF16 ? 2 : 4, &L,
+                   (flags & KVCR_CACHE_FP8_K) != 0))
+    return 0;
+  return L.total;
+}
+
 size_t kv_cache_storage_bytes_aux(int sinks, int window, int aux_frames, int tokens_per_frame,
                                   int heads, int head_dim, int chunk_frames, int with_rope,
                                   kvcr_dtype dtype) {
-  if (dtype != KVCR_BF16 && dtype != KVCR_F32) return 0;
-  StorageLayout L;
-  if (!make_layout(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
-                   with_rope != 0, dtype == KVCR_BF16 ? 2 : 4, &L))
-    return 0;
-  return L.total;
+  return kv_cache_storage_bytes_ex(sinks, window, aux_frames, tokens_per_frame, heads, head_dim,
+                                   chunk_frames, with_rope, dtype, 0u);
 }
 
 size_t kv_cache_storage_bytes(int sinks, int window, int tokens_per_frame, int heads, int head_dim,
@@ -338,11 +405,23 @@ int kv_cache_init_aux(kvcr_cache** out, int sinks, int window, int aux_frames,
                       int tokens_per_frame, int heads, int head_dim, int chunk_frames,
                       const kvcr_rope* rope, kvcr_dtype dtype, void* device_storage,
                       size_t storage_bytes) {
+  return kv_cache_init_ex(out, sinks, window, aux_frames, tokens_per_frame, heads, head_dim,
+                          chunk_frames, rope, dtype, 0u, device_storage, storage_bytes);
+}
+
+int kv_cache_init_ex(kvcr_cache** out, int sinks, int window, int aux_frames,
+                     int tokens_per_frame, int heads, int head_dim, int chunk_frames,
+                     const kvcr_rope* rope, kvcr_dtype dtype, unsigned flags,
+                     void* device_storage, size_t storage_bytes) {
   if (out == nullptr) return fail(KVCR_EINVAL, "kv_cache_init: out is NULL");
   *out = nullptr;
   if (dtype != KVCR_BF16 && dtype != KVCR_F32) return fail(KVCR_EINVAL, "kv_cache_init: bad dtype");
   if (head_dim != 64 && head_dim != 128)
     return fail(KVCR_EUNSUPPORTED, "kv_cache_init: head_dim must be 64 or 128");
+  if (flags & ~(unsigned)KVCR_CACHE_FP8_K) return fail(KVCR_EINVAL, "kv_cache_init: unknown flags");
+  const bool fp8 = (flags & KVCR_CACHE_FP8_K) != 0;
+  if (fp8 && (dtype != KVCR_BF16 || head_dim != 128))
+    return fail(KVCR_EUNSUPPORTED, "kv_cache_init: e4m3 K copies need bf16 and head_dim 128");
   if (sinks < 0 || window < 0 || aux_frames < 0 || sinks + window < 1 ||
       sinks + window + aux_frames > kMaxSlots)
     return fail(KVCR_ESHAPE,
@@ -365,7 +444,7 @@ int kv_cache_init_aux(kvcr_cache** out, int sinks, int window, int aux_frames,
   const size_t esize = dtype == KVCR_BF16 ? 2 : 4;
   StorageLayout L;
   if (!make_layout(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
-                   rope != nullptr, esize, &L))
+                   rope != nullptr, esize, &L, fp8))
     return fail(KVCR_ESHAPE, "kv_cache_init: bad sizes");
   const bool has_storage = device_storage != nullptr;
   if (!has_storage && storage_bytes != 0)
@@ -399,6 +478,7 @@ int kv_cache_init_aux(kvcr_cache** out, int sinks, int window, int aux_frames,
   c->lay = L;
   c->n_sm = n_sm;
   c->cc_major = cc;
+  c->fp8 = fp8;
   c->slot_frame.assign(sinks + window, -1);
   c->n_sinks_filled = 0;
   c->last_frame = -1;
@@ -432,6 +512,7 @@ int kv_cache_init_aux(kvcr_cache** out, int sinks, int window, int aux_frames,
                                 (uint64_t)(sinks + window + aux_frames)};
       int rc = encode_bf16_map(&c->tm_kc, c->storage + L.k_off, 4, dims, kKeyTile);
       if (!rc) rc = encode_bf16_map(&c->tm_vc, c->storage + L.v_off, 4, dims, kKeyTile);
+      if (!rc && fp8) rc = encode_map(&c->tm_kc8, true, c->storage + L.k8_off, 4, dims, kKeyTile);
       if (rc) {
         delete c;
         return rc;
@@ -480,12 +561,14 @@ int kv_cache_append_rope(kvcr_cache* c, const void* k, const void* v, const int3
     const long long frame_elems = (long long)c->T * c->H * c->D;
     int n = 0;
     std::vector<int32_t> written;
+    std::vector<int> written_slots;
     for (int i = 0; i < n_frames; ++i) {
       // skip frames not retained, or evicted again by a later frame of this call
       if (slots[i] < 0 || c->slot_frame[slots[i]] != frame_idx[i]) continue;
       p.dst_frame_off[n] = (long long)slots[i] * frame_elems;
       p.src_frame[n] = i;
       written.push_back(frame_idx[i]);
+      written_slots.push_back(slots[i]);
       ++n;
     }
     p.n_frames = n;
@@ -496,6 +579,7 @@ int kv_cache_append_rope(kvcr_cache* c, const void* k, const void* v, const int3
       LaunchScope scope(KVCR_K_APPEND_ROPE, s);
       e = launch_rope_copy(p, c->dtype, s, c->n_sm);
     }
+    if (e == cudaSuccess) e = quant_slots(c, written_slots, s);
     if (e != cudaSuccess) {
       restore(c, before);
       return cuda_fail(e, "kv_cache_append_rope: launch");
@@ -577,11 +661,17 @@ int kv_cache_append_rope_batch(kvcr_cache* const* caches, int n_caches, const vo
         }
     const size_t frame_bytes = (size_t)c0->T * c0->H * c0->D * c0->esize;
     int n = 0;
+    std::unique_ptr<QuantParams> qp(new QuantParams());
+    std::memset(qp.get(), 0, sizeof(QuantParams));
     for (int i = 0; i < n_caches; ++i) {
       const kvcr_cache* c = caches[i];
       for (int f = 0; f < n_frames; ++f) {
         // skip frames not retained, or evicted again by a later frame of this call
         if (slots[i][f] < 0 || c->slot_frame[slots[i][f]] != frame_idx[f]) continue;
+        if (c->fp8) {                              // its e4m3 copy, after the batch
+          quant_segment_of_slot(c, slots[i][f], *qp, qp->n_seg, qp->n_seg * blocks_of(c->T));
+          ++qp->n_seg;
+        }
         p->src_a[n] = static_cast<const uint8_t*>(k[i]) + (size_t)f * frame_bytes;
         p->src_b[n] = static_cast<const uint8_t*>(v[i]) + (size_t)f * frame_bytes;
         p->dst_a[n] = c->storage + c->lay.k_off + (size_t)slots[i][f] * frame_bytes;
@@ -598,6 +688,11 @@ int kv_cache_append_rope_batch(kvcr_cache* const* caches, int n_caches, const vo
       e = launch_rope_copy_batch(*p, c0->dtype, s, c0->n_sm);
     }
     delete p;
+    if (e == cudaSuccess && qp->n_seg > 0) {
+      qp->H = c0->H;
+      LaunchScope scope(KVCR_K_QUANT_E4M3, s);
+      e = launch_quant_e4m3(*qp, c0->D, s);
+    }
     if (e != cudaSuccess) {
       for (int i = 0; i < n_caches; ++i) restore(caches[i], before[i]);
       return cuda_fail(e, "kv_cache_append_rope_batch: launch");
@@ -668,6 +763,20 @@ int kv_cache_slot_data(const kvcr_cache* c, int slot, const void** k, const void
   return KVCR_OK;
 }
 
+int kv_cache_slot_data_fp8(const kvcr_cache* c, int slot, const void** k_codes,
+                           const float** k_scales) {
+  if (c == nullptr || k_codes == nullptr || k_scales == nullptr)
+    return fail(KVCR_EINVAL, "kv_cache_slot_data_fp8: NULL");
+  if (!c->has_storage || !c->fp8)
+    return fail(KVCR_ESTATE, "kv_cache_slot_data_fp8: the cache keeps no e4m3 K copies");
+  if (slot < 0 || slot >= c->S + c->W + c->A)
+    return fail(KVCR_EINVAL, "kv_cache_slot_data_fp8: bad slot");
+  *k_codes = c->storage + c->lay.k8_off + (size_t)slot * c->T * c->H * c->D;
+  *k_scales = reinterpret_cast<const float*>(c->storage + c->lay.k8s_off) +
+              (size_t)slot * blocks_of(c->T) * c->H;
+  return KVCR_OK;
+}
+
 int kv_cache_set_aux(kvcr_cache* c, const void* k, const void* v, const int32_t* aux_pos,
                      int n_frames, void* stream) {
   const char* fn = "kv_cache_set_aux";
@@ -706,6 +815,11 @@ int kv_cache_set_aux(kvcr_cache* c, const void* k, const void* v, const int32_t*
     {
       LaunchScope scope(KVCR_K_SET_AUX, s);
       e = launch_rope_copy(p, c->dtype, s, c->n_sm);
+    }
+    if (e == cudaSuccess && c->fp8) {
+      std::vector<int> aux_slots;
+      for (int f = 0; f < n_frames; ++f) aux_slots.push_back(c->S + c->W + f);
+      e = quant_slots(c, aux_slots, s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "kv_cache_set_aux: launch");
   }
@@ -834,6 +948,133 @@ int chunk_attention_fwd(kvcr_cache* c, const void* q, int n_q, const void* k_cur
     }
     if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd: fp32 attention launch");
   }
+  return KVCR_OK;
+}
+
+// ============================================== chunk attention, e4m3 QK^T
+// Stage (RoPE) as chunk_attention_fwd(), quantize the staged queries and current
+// keys to e4m3 blocks of 128 tokens, then the tensor-core kernel with the QK^T
+// product in e4m3 over the cache's e4m3 K copies and the P V product in bf16.
+int chunk_attention_fwd_fp8(kvcr_cache* c, const void* q, int n_q, const void* k_cur,
+                            const void* v_cur, const int32_t* cur_frame_idx, int n_cur_frames,
+                            float softmax_scale, void* o, float* lse, void* stream) {
+  const char* fn = "chunk_attention_fwd_fp8";
+  if (c == nullptr) return fail(KVCR_EINVAL, std::string(fn) + ": cache is NULL");
+  if (!c->has_storage) return fail(KVCR_ESTATE, std::string(fn) + ": bookkeeping-only cache");
+  if (!c->fp8)
+    return fail(KVCR_ESTATE, std::string(fn) + ": the cache keeps no e4m3 K copies "
+                                               "(create it with KVCR_CACHE_FP8_K)");
+  if (n_cur_frames < 1 || n_cur_frames > c->F)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_cur_frames must be in [1, chunk_frames]");
+  if (n_q < 0) return fail(KVCR_ESHAPE, std::string(fn) + ": n_q < 0");
+  const int n_cur = n_cur_frames * c->T;
+  if (c->rope && n_q != n_cur)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": with RoPE n_q must be n_cur_frames * T");
+  if (!c->rope && (long long)n_q > (long long)c->F * c->T)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_q larger than the query staging "
+                                               "(chunk_frames * tokens_per_frame)");
+  int rc = check_frames(c, cur_frame_idx, n_cur_frames, fn);
+  if (rc) return rc;
+  if (n_q == 0) return KVCR_OK;
+  if (!q || !k_cur || !v_cur || !o) return fail(KVCR_EINVAL, std::string(fn) + ": NULL tensor");
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(o))
+    return fail(KVCR_EINVAL, std::string(fn) + ": tensors must be 16-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(KVCR_EINVAL, std::string(fn) + ": lse must be 4-byte aligned");
+  if ((long long)n_q * c->H * c->D > (1LL << 31) - 1)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_q too large");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)c->D);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  int slots[kMaxSlots];
+  int n_vis = 0;
+  for (int i = 0; i < c->S + c->W; ++i)
+    if (c->slot_frame[i] >= 0) slots[n_vis++] = i;
+  for (int i = 0; i < c->n_aux; ++i) slots[n_vis++] = c->S + c->W + i;  // auxiliary frames
+
+  const void* q_src = q;
+  const void* k_src = k_cur;
+  cudaError_t e;
+  if (c->rope) {
+    RopeCopyParams p;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(c, p);
+    p.src_a = q;
+    p.src_b = k_cur;
+    p.dst_a = c->storage + c->lay.q_off;
+    p.dst_b = c->storage + c->lay.ks_off;
+    p.rotate_a = 1;
+    p.rotate_b = 1;
+    p.n_frames = n_cur_frames;
+    const long long frame_elems = (long long)c->T * c->H * c->D;
+    for (int f = 0; f < n_cur_frames; ++f) {
+      p.dst_frame_off[f] = f * frame_elems;
+      p.src_frame[f] = f;
+    }
+    fill_ttab(c, p, cur_frame_idx, n_cur_frames);
+    {
+      LaunchScope scope(KVCR_K_ROPE_STAGE, s);
+      e = launch_rope_copy(p, c->dtype, s, c->n_sm);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd_fp8: rope stage launch");
+    q_src = c->storage + c->lay.q_off;
+    k_src = c->storage + c->lay.ks_off;
+  }
+  uint8_t* q8 = c->storage + c->lay.q8_off;
+  uint8_t* k8 = c->storage + c->lay.c8_off;
+  float* q8s = reinterpret_cast<float*>(c->storage + c->lay.q8s_off);
+  float* k8s = reinterpret_cast<float*>(c->storage + c->lay.c8s_off);
+  {
+    std::unique_ptr<QuantParams> qp(new QuantParams());
+    std::memset(qp.get(), 0, sizeof(QuantParams));
+    qp->src[0] = q_src;
+    qp->dst[0] = q8;
+    qp->scale[0] = q8s;
+    qp->n_tok[0] = n_q;
+    qp->tile0[0] = 0;
+    qp->src[1] = k_src;
+    qp->dst[1] = k8;
+    qp->scale[1] = k8s;
+    qp->n_tok[1] = n_cur;
+    qp->tile0[1] = blocks_of(n_q);
+    qp->n_seg = 2;
+    qp->H = c->H;
+    LaunchScope scope(KVCR_K_QUANT_E4M3, s);
+    e = launch_quant_e4m3(*qp, c->D, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd_fp8: quantization launch");
+
+  ChunkAttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint64_t dq[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_q};
+  const uint64_t dn[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_cur};
+  rc = encode_map(&p.tm_q, true, q8, 3, dq, kTile);
+  if (!rc) rc = encode_map(&p.tm_kn, true, k8, 3, dn, kKeyTile);
+  if (!rc) rc = encode_bf16_map(&p.tm_vn, v_cur, 3, dn, kKeyTile);
+  if (rc) return rc;
+  p.tm_kc = c->tm_kc8;
+  p.tm_vc = c->tm_vc;
+  p.q_scale = q8s;
+  p.kc_scale = reinterpret_cast<const float*>(c->storage + c->lay.k8s_off);
+  p.kn_scale = k8s;
+  p.c.o = o;
+  p.c.lse = lse;
+  p.c.n_q = n_q;
+  p.c.H = c->H;
+  p.c.scale_log2 = (float)(scale * 1.4426950408889634);
+  p.c.inject = inject_state().kind;
+  p.c.wait_ns = inject_state().wait_ns;
+  p.s.T = c->T;
+  p.s.n_vis = n_vis;
+  p.s.tiles_per_slot = (c->T + kKeyTile - 1) / kKeyTile;
+  p.s.n_cur = n_cur;
+  p.s.cur_tiles = (n_cur + kKeyTile - 1) / kKeyTile;
+  for (int i = 0; i < n_vis; ++i) p.s.slots[i] = slots[i];
+  {
+    LaunchScope scope(KVCR_K_CHUNK_ATTN_FP8, s);
+    e = launch_chunk_attn_sm100(p, c->D, (n_q + kTile - 1) / kTile, s, true);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd_fp8: attention launch");
   return KVCR_OK;
 }
 

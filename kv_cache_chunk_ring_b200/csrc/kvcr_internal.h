@@ -82,6 +82,11 @@ struct ChunkAttnParams {
   CUtensorMap tm_vn;  // 3D current V
   AttnCommon c;
   ChunkSched s;
+  // e4m3 QK^T only (tm_q, tm_kc, tm_kn then map the e4m3 codes): scale of each
+  // 128-token block and head, [block][H] (cached keys: [slot][block][H])
+  const float* q_scale;
+  const float* kc_scale;
+  const float* kn_scale;
 };
 
 struct MobaAttnParams {
@@ -93,7 +98,7 @@ struct MobaAttnParams {
 };
 
 cudaError_t launch_chunk_attn_sm100(const ChunkAttnParams& p, int head_dim, int n_q_tiles,
-                                    cudaStream_t s);
+                                    cudaStream_t s, bool qk_e4m3 = false);
 cudaError_t launch_moba_attn_sm100(const MobaAttnParams& p, int head_dim, cudaStream_t s);
 
 // fp32 CUDA-core attention over the same key sequence (cached slots + current)
@@ -110,6 +115,21 @@ struct F32AttnParams {
   int slots[kMaxSlots];
 };
 cudaError_t launch_attn_f32(const F32AttnParams& p, cudaStream_t s);
+
+// ------------------------------------------------- e4m3 block quantization --
+// Segment i: src[i] bf16 [n_tok[i]][H][D] -> dst[i] e4m3 codes (same layout, one
+// byte each) and scale[i] fp32 [ceil(n_tok[i] / 128)][H]; the blocks of segment i
+// are grid blocks tile0[i] .. tile0[i] + ceil(n_tok[i] / 128) - 1.
+constexpr int kMaxQuantSegs = 256;
+struct QuantParams {
+  const void* src[kMaxQuantSegs];
+  void* dst[kMaxQuantSegs];
+  float* scale[kMaxQuantSegs];
+  int n_tok[kMaxQuantSegs];
+  int tile0[kMaxQuantSegs];
+  int n_seg, H;
+};
+cudaError_t launch_quant_e4m3(const QuantParams& p, int head_dim, cudaStream_t s);
 
 // device status words (one per kernel translation unit)
 cudaError_t read_and_clear_status_attn(int* st, cudaStream_t s);

@@ -21,18 +21,22 @@ KVCR_OK, KVCR_EINVAL, KVCR_ESHAPE, KVCR_ESTATE = 0, -1, -2, -3
 KVCR_ECUDA, KVCR_ETIMEOUT, KVCR_ESTORAGE, KVCR_EUNSUPPORTED = -4, -5, -6, -7
 KVCR_BF16, KVCR_F32 = 0, 1
 KVCR_TILE_EMPTY, KVCR_TILE_PARTIAL, KVCR_TILE_FULL = 0, 1, 2
+KVCR_CACHE_FP8_K = 1
 (KVCR_K_APPEND_ROPE, KVCR_K_ROPE_STAGE, KVCR_K_CHUNK_ATTN, KVCR_K_MOBA_ATTN,
  KVCR_K_ATTN_F32, KVCR_K_MOBA_BWD_PREP, KVCR_K_MOBA_BWD_DKDV, KVCR_K_MOBA_BWD_DQ,
- KVCR_K_SET_AUX, KVCR_K_APPEND_BATCH) = range(10)
+ KVCR_K_SET_AUX, KVCR_K_APPEND_BATCH, KVCR_K_QUANT_E4M3, KVCR_K_CHUNK_ATTN_FP8) = range(12)
 KERNEL_NAMES = {KVCR_K_APPEND_ROPE: "append_rope", KVCR_K_ROPE_STAGE: "rope_stage",
                 KVCR_K_CHUNK_ATTN: "chunk_attn", KVCR_K_MOBA_ATTN: "moba_attn",
                 KVCR_K_ATTN_F32: "attn_f32", KVCR_K_MOBA_BWD_PREP: "moba_bwd_prep",
                 KVCR_K_MOBA_BWD_DKDV: "moba_bwd_dkdv", KVCR_K_MOBA_BWD_DQ: "moba_bwd_dq",
-                KVCR_K_SET_AUX: "set_aux", KVCR_K_APPEND_BATCH: "append_batch"}
+                KVCR_K_SET_AUX: "set_aux", KVCR_K_APPEND_BATCH: "append_batch",
+                KVCR_K_QUANT_E4M3: "quant_e4m3", KVCR_K_CHUNK_ATTN_FP8: "chunk_attn_fp8"}
 
 # every symbol include/kvcr.h declares
 EXPORTS = [
     "kv_cache_storage_bytes", "kv_cache_init", "kv_cache_storage_bytes_aux", "kv_cache_init_aux",
+    "kv_cache_storage_bytes_ex", "kv_cache_init_ex", "kv_cache_slot_data_fp8",
+    "chunk_attention_fwd_fp8",
     "kv_cache_set_aux", "kv_cache_num_aux", "kv_cache_append_rope", "kv_cache_append_rope_batch",
     "kv_cache_evict",
     "kv_cache_slot_map", "kv_cache_last_append", "kv_cache_num_cached", "kv_cache_slot_data",
@@ -169,6 +173,13 @@ def lib() -> ctypes.CDLL:
         "kv_cache_storage_bytes_aux": (c_sz, [c_int] * 8 + [c_int]),
         "kv_cache_init_aux": (c_int, [ctypes.POINTER(c_p), c_int, c_int, c_int, c_int, c_int, c_int,
                                       c_int, ctypes.POINTER(kvcr_rope), c_int, c_p, c_sz]),
+        "kv_cache_storage_bytes_ex": (c_sz, [c_int] * 9 + [ctypes.c_uint]),
+        "kv_cache_init_ex": (c_int, [ctypes.POINTER(c_p), c_int, c_int, c_int, c_int, c_int, c_int,
+                                     c_int, ctypes.POINTER(kvcr_rope), c_int, ctypes.c_uint, c_p,
+                                     c_sz]),
+        "kv_cache_slot_data_fp8": (c_int, [c_p, c_int, ctypes.POINTER(c_p), ctypes.POINTER(c_p)]),
+        "chunk_attention_fwd_fp8": (c_int, [c_p, c_p, c_int, c_p, c_p, i32p, c_int, c_f, c_p, c_p,
+                                            c_p]),
         "kv_cache_set_aux": (c_int, [c_p, c_p, c_p, i32p, c_int, c_p]),
         "kv_cache_num_aux": (c_int, [c_p, ctypes.POINTER(c_int)]),
         "kv_cache_append_rope": (c_int, [c_p, c_p, c_p, i32p, c_int, c_p]),
@@ -257,6 +268,21 @@ def kv_cache_storage_bytes_aux(sinks, window, aux_frames, tokens_per_frame, head
 def kv_cache_init_aux(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
                       rope, dtype, storage) -> ctypes.c_void_p:
     """Create a cache with ``aux_frames`` auxiliary slots over ``storage``."""
+    return kv_cache_init_ex(sinks, window, aux_frames, tokens_per_frame, heads, head_dim,
+                            chunk_frames, rope, dtype, 0, storage)
+
+
+def kv_cache_storage_bytes_ex(sinks, window, aux_frames, tokens_per_frame, heads, head_dim,
+                              chunk_frames, with_rope, dtype, flags) -> int:
+    return int(lib().kv_cache_storage_bytes_ex(sinks, window, aux_frames, tokens_per_frame, heads,
+                                               head_dim, chunk_frames, int(bool(with_rope)),
+                                               _dtype_code(dtype), int(flags)))
+
+
+def kv_cache_init_ex(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
+                     rope, dtype, flags, storage) -> ctypes.c_void_p:
+    """Create a cache with ``aux_frames`` auxiliary slots and cache ``flags``
+    (KVCR_CACHE_FP8_K) over ``storage``."""
     h = ctypes.c_void_p()
     rp = None
     if rope is not None:
@@ -264,9 +290,9 @@ def kv_cache_init_aux(sinks, window, aux_frames, tokens_per_frame, heads, head_d
                                     rope.pairs_w, float(rope.base)))
     ptr = None if storage is None else storage.data_ptr()
     nbytes = 0 if storage is None else storage.numel() * storage.element_size()
-    _check(lib().kv_cache_init_aux(ctypes.byref(h), sinks, window, aux_frames, tokens_per_frame,
-                                   heads, head_dim, chunk_frames, rp, _dtype_code(dtype), ptr,
-                                   nbytes))
+    _check(lib().kv_cache_init_ex(ctypes.byref(h), sinks, window, aux_frames, tokens_per_frame,
+                                  heads, head_dim, chunk_frames, rp, _dtype_code(dtype),
+                                  int(flags), ptr, nbytes))
     _CACHE_INFO[h.value] = (tokens_per_frame, heads, head_dim, _dtype_code(dtype),
                             rope is not None)
     return h
@@ -387,6 +413,24 @@ def chunk_attention_fwd(handle, q, k_cur, v_cur, cur_frame_idx: Sequence[int], o
                                      float(softmax_scale), _ptr(o), _ptr(lse), _stream(stream)))
 
 
+def chunk_attention_fwd_fp8(handle, q, k_cur, v_cur, cur_frame_idx: Sequence[int], o, lse=None,
+                            softmax_scale: float = 0.0, stream=None) -> None:
+    """chunk_attention_fwd with the QK^T product in e4m3 (cache made with KVCR_CACHE_FP8_K)."""
+    _check_chunk_args(handle, q, k_cur, v_cur, len(cur_frame_idx), o, lse)
+    _check(lib().chunk_attention_fwd_fp8(handle, _ptr(q), q.shape[0], _ptr(k_cur), _ptr(v_cur),
+                                         _i32(cur_frame_idx), len(cur_frame_idx),
+                                         float(softmax_scale), _ptr(o), _ptr(lse),
+                                         _stream(stream)))
+
+
+def kv_cache_slot_data_fp8(handle, slot: int) -> Tuple[int, int]:
+    """Device addresses (ints) of one slot's e4m3 K codes and block scales."""
+    k = ctypes.c_void_p()
+    sc = ctypes.c_void_p()
+    _check(lib().kv_cache_slot_data_fp8(handle, slot, ctypes.byref(k), ctypes.byref(sc)))
+    return int(k.value), int(sc.value)
+
+
 def chunk_attention_fwd_static_scratch(handle, q, k_cur, v_cur, cur_frame_idx: Sequence[int], o,
                                        lse=None, softmax_scale: float = 0.0,
                                        stream=None) -> None:
@@ -483,23 +527,24 @@ class Cache:
 
     def __init__(self, sinks: int, window: int, tokens_per_frame: int, heads: int, head_dim: int,
                  chunk_frames: int, rope=None, dtype="bf16", device="cuda",
-                 bookkeeping_only: bool = False, aux_frames: int = 0):
+                 bookkeeping_only: bool = False, aux_frames: int = 0, fp8_k: bool = False):
         self.sinks, self.window, self.aux_frames = sinks, window, aux_frames
+        self.flags = KVCR_CACHE_FP8_K if fp8_k else 0
         self.T, self.H, self.D, self.F = tokens_per_frame, heads, head_dim, chunk_frames
         self.rope = rope
         self.dtype_code = _dtype_code(dtype)
         self.storage = None
         if not bookkeeping_only:
             import torch
-            nbytes = kv_cache_storage_bytes_aux(sinks, window, aux_frames, tokens_per_frame, heads,
-                                                head_dim, chunk_frames, rope is not None,
-                                                self.dtype_code)
+            nbytes = kv_cache_storage_bytes_ex(sinks, window, aux_frames, tokens_per_frame, heads,
+                                               head_dim, chunk_frames, rope is not None,
+                                               self.dtype_code, self.flags)
             if nbytes == 0:
                 raise KvcrError(KVCR_ESHAPE, "invalid cache sizes")
             self.storage = torch.empty(nbytes, dtype=torch.uint8, device=device)
-        self.handle = kv_cache_init_aux(sinks, window, aux_frames, tokens_per_frame, heads,
-                                        head_dim, chunk_frames, rope, self.dtype_code,
-                                        self.storage)
+        self.handle = kv_cache_init_ex(sinks, window, aux_frames, tokens_per_frame, heads,
+                                       head_dim, chunk_frames, rope, self.dtype_code, self.flags,
+                                       self.storage)
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -554,14 +599,28 @@ class Cache:
         return k, v
 
     def attention(self, q, k_cur, v_cur, frames: Sequence[int], want_lse: bool = False,
-                  out=None, softmax_scale: float = 0.0, stream=None):
+                  out=None, softmax_scale: float = 0.0, stream=None, fp8: bool = False):
+        """Chunk attention (``fp8``: the e4m3 QK^T variant, cache made with fp8_k)."""
         import torch
         o = out if out is not None else torch.empty_like(q)
         lse = None
         if want_lse:
             lse = torch.empty((self.H, q.shape[0]), dtype=torch.float32, device=q.device)
-        chunk_attention_fwd(self.handle, q, k_cur, v_cur, frames, o, lse, softmax_scale, stream)
+        fn = chunk_attention_fwd_fp8 if fp8 else chunk_attention_fwd
+        fn(self.handle, q, k_cur, v_cur, frames, o, lse, softmax_scale, stream)
         return o, lse
+
+    def slot_tensors_fp8(self, slot: int):
+        """Views (torch) of one slot's e4m3 K codes [T, H, D] (uint8) and block scales
+        [ceil(T / 128), H] (fp32)."""
+        kp, sp = kv_cache_slot_data_fp8(self.handle, slot)
+        base = self.storage.data_ptr()
+        n = self.T * self.H * self.D
+        nb = (self.T + 127) // 128
+        codes = self.storage[kp - base:kp - base + n].view(self.T, self.H, self.D)
+        scales = self.storage[sp - base:sp - base + 4 * nb * self.H].view(
+            __import__("torch").float32).view(nb, self.H)
+        return codes, scales
 
 
 def default_scale(head_dim: int) -> float:

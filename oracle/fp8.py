@@ -21,7 +21,11 @@ own speed lever on this path; here the 8-bit format is the tensor cores' e4m3):
 Readings: the block is 128 tokens x one head (the kernel's tile), the fp32
 steps are written out so that a kernel taking the same steps makes the same
 integer decisions (the code of every element), and V stays in bf16 (the
-pages quantize only QK^T).
+pages quantize only QK^T).  In the chunk rollout what is quantized is the
+tensor the bf16 path would hold: RoPE'd Q and K rounded once to bf16
+(``round_bf16``); the blocks follow the attention's tiles -- 128 consecutive
+tokens of one cached (or auxiliary) frame, 128 consecutive tokens of the
+current chunk for its own queries and keys (``fp8_operand``).
 
 Parity: pinned (every finite code rounds to itself; ties to even; agreement
 with torch's float8_e4m3fn conversion below the saturation point; the
@@ -97,6 +101,23 @@ def dequantize_blocks(codes, scales, rows: int = 128) -> np.ndarray:
     codes = np.asarray(codes, dtype=np.float64)
     s = np.repeat(np.asarray(scales, dtype=np.float64), rows, axis=0)[:codes.shape[0]]
     return codes * s[:, :, None]
+
+
+def round_bf16(x) -> np.ndarray:
+    """Round to the nearest bf16 value (8 significant bits, ties to the even
+    significand; spacing 2^-133 below the normal range); float64 out."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)                           # 2^(e-1) <= |x| < 2^e
+    q = np.maximum(e - 8, -133).astype(np.float64)
+    step = np.exp2(q)
+    return np.where(x == 0, x, np.rint(x / step) * step)
+
+
+def fp8_operand(x, rows: int = 128) -> np.ndarray:
+    """What the low-precision product sees of a [L, H, D] operand: x rounded to bf16,
+    block-quantized to e4m3 per 128 rows and head, dequantized (float64)."""
+    codes, scales = quantize_blocks(round_bf16(x), rows)
+    return dequantize_blocks(codes, scales, rows)
 
 
 def attention_fp8_qk(q, k, v, scale: float, rows: int = 128):

@@ -39,6 +39,7 @@ from typing import Dict, List, Optional
 
 import numpy as np
 
+from . import fp8
 from .attn import attention
 from .cache import CacheModel
 from .rope import rope3d, rope_pairs_default, rope_positions
@@ -57,14 +58,17 @@ class RolloutResult:
 
 
 def rollout(spec, chunks, rows_for=None, use_rope: bool = True,
-            window_schedule: Optional[List[int]] = None, aux_for=None) -> RolloutResult:
+            window_schedule: Optional[List[int]] = None, aux_for=None,
+            qk_fp8: bool = False) -> RolloutResult:
     """Run the rollout of ``spec`` (a RolloutSpec) over ``chunks``.
 
     ``chunks`` yields dicts with chunk, step, frames, q, k, v as produced by
     ``workloads.rollout_chunks``.  ``rows_for(chunk, step)`` returns the query
     rows to evaluate (default: all).  ``aux_for(chunk)`` returns None or
     (k_aux, v_aux, positions) with k_aux, v_aux [n * T, H, D] and positions a
-    list of n temporal positions or None.
+    list of n temporal positions or None.  ``qk_fp8``: the QK^T product sees Q
+    and K as ``fp8.fp8_operand`` gives them -- blocks of 128 tokens of each
+    cached or auxiliary frame, and of the current chunk for its own Q and K.
     """
     T = spec.grid_h * spec.grid_w
     scale = 1.0 / math.sqrt(spec.head_dim)
@@ -88,7 +92,15 @@ def rollout(spec, chunks, rows_for=None, use_rope: bool = True,
             for f in pending_evicted:
                 store.pop(f, None)
         rows = np.arange(q.shape[0]) if rows_for is None else np.asarray(rows_for(c, s))
-        if use_rope:
+        if qk_fp8:
+            # a query block's scale depends on all of its rows: rotate them all
+            if use_rope:
+                t, hh, ww = rope_positions(frames, spec.grid_h, spec.grid_w)
+                q_rot = fp8.fp8_operand(rope3d(q, t, hh, ww, pairs, spec.rope().base))[rows]
+                k_rot = rope3d(k, t, hh, ww, pairs, spec.rope().base)
+            else:
+                q_rot, k_rot = fp8.fp8_operand(q)[rows], k
+        elif use_rope:
             # each token turns by the angles of its own position, so only the
             # evaluated query rows need rotating
             t, hh, ww = rope_positions(frames, spec.grid_h, spec.grid_w)
@@ -106,7 +118,14 @@ def rollout(spec, chunks, rows_for=None, use_rope: bool = True,
                 ta, ha, wa = rope_positions(list(aux[2]), spec.grid_h, spec.grid_w)
                 ka = rope3d(ka, ta, ha, wa, pairs, spec.rope().base)
             k_aux, v_aux = [ka], [va]
-        k_all = np.concatenate([store[f][0] for f in vis] + k_aux + [k_rot], axis=0)
+        if qk_fp8:
+            # per frame for cached and auxiliary keys, over the chunk for its own
+            k_cached = [fp8.fp8_operand(store[f][0]) for f in vis]
+            k_aux = [fp8.fp8_operand(ka[n * T:(n + 1) * T]) for ka in k_aux
+                     for n in range(ka.shape[0] // T)]
+            k_all = np.concatenate(k_cached + k_aux + [fp8.fp8_operand(k_rot)], axis=0)
+        else:
+            k_all = np.concatenate([store[f][0] for f in vis] + k_aux + [k_rot], axis=0)
         v_all = np.concatenate([store[f][1] for f in vis] + v_aux + [v], axis=0)
         o, lse = attention(q_rot, k_all, v_all, scale)
         res.outputs.append(o)
