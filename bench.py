@@ -371,6 +371,14 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
         "append_hbm_frac": round(app_gbs / float(peaks["hbm_gbs"]), 4),
         "clocks": clocks,
     }
+    # the same kernel against the tensor cores' issue rate at the SM clock seen during the
+    # timed region: 148 SMs x 8192 dense bf16 FLOP per SM clock (one 128 x 128 x 16 MMA
+    # per 32 clocks, measured full-rate in a standalone tcgen05 loop)
+    if clocks and clocks.get("sm_mhz"):
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        clock_peak = n_sm * 8192 * clocks["sm_mhz"] * 1e6 / 1e12
+        out["attn_kernel_frac_of_clock_peak"] = round(achieved / clock_peak, 4)
+        out["clock_peak_tflops"] = round(clock_peak, 1)
     return out
 
 

@@ -161,15 +161,22 @@ enum {
      * it with one fp32 scale per block of 128 tokens and head, written by the same
      * append / set_aux call; chunk_attention_fwd_fp8() reads it.  Needs bf16 and
      * head_dim 128. */
-    KVCR_CACHE_FP8_K = 1
+    KVCR_CACHE_FP8_K = 1,
+    /* Keep chunk_frames spare frame slots so that chunk_attention_fwd_finalize()
+     * can write the chunk's rotated K and its V straight into cache storage while
+     * the frames they replace are still read (see there).  bf16 caches. */
+    KVCR_CACHE_FUSED_FINALIZE = 2
 };
 
-/* kv_cache_storage_bytes_aux() / kv_cache_init_aux() with cache flags (0 or
- * KVCR_CACHE_FP8_K).  With KVCR_CACHE_FP8_K the storage also holds the e4m3 K
- * copies (T * H * D bytes per frame slot), their scales (4 * ceil(T / 128) * H
- * bytes per slot) and the e4m3 staging of one chunk's queries and keys.
- * kv_cache_init_ex returns KVCR_EUNSUPPORTED for KVCR_CACHE_FP8_K with fp32 or
- * head_dim 64, KVCR_EINVAL for unknown flags. */
+/* kv_cache_storage_bytes_aux() / kv_cache_init_aux() with cache flags (0,
+ * KVCR_CACHE_FP8_K or KVCR_CACHE_FUSED_FINALIZE, not both).  With
+ * KVCR_CACHE_FP8_K the storage also holds the e4m3 K copies (T * H * D bytes per
+ * frame slot), their scales (4 * ceil(T / 128) * H bytes per slot) and the e4m3
+ * staging of one chunk's queries and keys; with KVCR_CACHE_FUSED_FINALIZE,
+ * chunk_frames more K / V frame slots (sinks + window + aux_frames + chunk_frames
+ * <= 32).  kv_cache_init_ex returns KVCR_EUNSUPPORTED for KVCR_CACHE_FP8_K with
+ * fp32 or head_dim 64 and for KVCR_CACHE_FUSED_FINALIZE with fp32, KVCR_EINVAL
+ * for unknown or combined flags. */
 size_t kv_cache_storage_bytes_ex(int sinks, int window, int aux_frames, int tokens_per_frame,
                                  int heads, int head_dim, int chunk_frames, int with_rope,
                                  kvcr_dtype dtype, unsigned flags);
@@ -296,6 +303,26 @@ int chunk_attention_fwd_static_scratch(kvcr_cache *c, const void *q, int n_q,
                                        const void *k_cur, const void *v_cur,
                                        const int32_t *cur_frame_idx, int n_cur_frames,
                                        float softmax_scale, void *o, float *lse, void *stream);
+
+/* The last denoising step of a chunk: chunk_attention_fwd() followed by
+ * kv_cache_append_rope(k_cur, v_cur, cur_frame_idx), with one pass over the
+ * chunk's K and V.  The finalized states enter the retained slots ("Westlake AGI
+ * Lab's 'World in World' Steers Frozen Video Models", second paragraph) and the
+ * step that finalizes reads the frames they evict: here the chunk's rotated K
+ * and its V are written once, into spare frame slots, read from there by this
+ * call's attention as the current keys, and then become cached frames by
+ * relabelling (the slots of the frames they evict become the spare ones), so
+ * the separate append pass over K and V disappears.  Slot maps, eviction and
+ * the result of kv_cache_slot_data() are exactly those of the two-call
+ * sequence; outputs equal chunk_attention_fwd()'s up to the order of fp32
+ * accumulation (the chunk's keys are read frame by frame).  Needs a cache made
+ * with KVCR_CACHE_FUSED_FINALIZE (else KVCR_ESTATE).  Arguments and errors are
+ * those of chunk_attention_fwd() and kv_cache_append_rope(); on error nothing
+ * changes. */
+int chunk_attention_fwd_finalize(kvcr_cache *c, const void *q, int n_q, const void *k_cur,
+                                 const void *v_cur, const int32_t *cur_frame_idx,
+                                 int n_cur_frames, float softmax_scale, void *o, float *lse,
+                                 void *stream);
 
 /* chunk_attention_fwd() with the QK^T product in 8 bits: the pages' own speed
  * lever on this path is an 8-bit QK^T (kaarelkaarelson.com/lingbot, kernel table,

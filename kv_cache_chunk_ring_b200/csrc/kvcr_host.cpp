@@ -179,12 +179,13 @@ struct StorageLayout {
 int blocks_of(long long n) { return (int)((n + 127) / 128); }
 
 bool make_layout(int S, int W, int A, int T, int H, int D, int F, bool rope, size_t esize,
-                 StorageLayout* L, bool fp8 = false) {
-  if (S < 0 || W < 0 || A < 0 || S + W < 1 || S + W + A > kMaxSlots || T < 1 || H < 1 || D < 1 ||
+                 StorageLayout* L, bool fp8 = false, bool spare = false) {
+  const int n_phys = S + W + A + (spare ? F : 0);
+  if (S < 0 || W < 0 || A < 0 || S + W < 1 || n_phys > kMaxSlots || T < 1 || H < 1 || D < 1 ||
       F < 1 || F > kMaxFrames)
     return false;
   const size_t frame = (size_t)T * H * D * esize;
-  const size_t slots = (size_t)(S + W + A);  // anchors, window, auxiliary
+  const size_t slots = (size_t)n_phys;  // anchors, window, auxiliary, spare
   size_t off = 0;
   L->k_off = off;
   off = align_up(off + slots * frame, 256);
@@ -241,6 +242,12 @@ struct kvcr_cache {
   CUtensorMap tm_kc, tm_vc;
   bool fp8;             // e4m3 K copies kept (KVCR_CACHE_FP8_K)
   CUtensorMap tm_kc8;   // 4D map over the e4m3 K copies
+  // Physical frame slot of each anchor / window slot (the identity unless
+  // chunk_attention_fwd_finalize() relabelled them) and the spare physical slots
+  // (KVCR_CACHE_FUSED_FINALIZE: chunk_frames of them, after the auxiliary slots).
+  bool fused;
+  std::vector<int> phys;
+  std::vector<int> spare;
   // slot table
   std::vector<int> slot_frame;
   int n_sinks_filled;
@@ -260,10 +267,11 @@ struct SlotState {
   int n_sinks_filled;
   std::deque<int> recent;
   int last_frame;
+  std::vector<int> phys, spare;
 };
 
 SlotState snapshot(const kvcr_cache* c) {
-  return SlotState{c->slot_frame, c->n_sinks_filled, c->recent, c->last_frame};
+  return SlotState{c->slot_frame, c->n_sinks_filled, c->recent, c->last_frame, c->phys, c->spare};
 }
 
 void restore(kvcr_cache* c, const SlotState& s) {
@@ -271,6 +279,24 @@ void restore(kvcr_cache* c, const SlotState& s) {
   c->n_sinks_filled = s.n_sinks_filled;
   c->recent = s.recent;
   c->last_frame = s.last_frame;
+  c->phys = s.phys;
+  c->spare = s.spare;
+}
+
+// Physical frame slot of a slot index (anchor / window slots through the
+// relabelling table, auxiliary slots as they are).
+int phys_of(const kvcr_cache* c, int slot) {
+  return slot < c->S + c->W ? c->phys[slot] : slot;
+}
+
+// Visible frames of the next attention call as physical slots: cached frames in
+// slot order, then the auxiliary frames.
+int visible_slots(const kvcr_cache* c, int* slots) {
+  int n = 0;
+  for (int i = 0; i < c->S + c->W; ++i)
+    if (c->slot_frame[i] >= 0) slots[n++] = c->phys[i];
+  for (int i = 0; i < c->n_aux; ++i) slots[n++] = c->S + c->W + i;
+  return n;
 }
 
 // Apply the slot rules to one frame; returns its slot (-1 = not retained) and
@@ -327,6 +353,7 @@ void fill_common(const kvcr_cache* c, RopeCopyParams& p) {
 // to its e4m3 copy and block scales.
 void quant_segment_of_slot(const kvcr_cache* c, int slot, QuantParams& p, int i, int tile0) {
   const size_t codes = (size_t)c->T * c->H * c->D;
+  slot = phys_of(c, slot);
   p.src[i] = c->storage + c->lay.k_off + (size_t)slot * codes * c->esize;
   p.dst[i] = c->storage + c->lay.k8_off + (size_t)slot * codes;
   p.scale[i] = reinterpret_cast<float*>(c->storage + c->lay.k8s_off) +
@@ -372,11 +399,12 @@ size_t kv_cache_storage_bytes_ex(int sinks, int window, int aux_frames, int toke
                                  int heads, int head_dim, int chunk_frames, int with_rope,
                                  kvcr_dtype dtype, unsigned flags) {
   if (dtype != KVCR_BF16 && dtype != KVCR_F32) return 0;
-  if (flags & ~(unsigned)KVCR_CACHE_FP8_K) return 0;
+  if (flags & ~(unsigned)(KVCR_CACHE_FP8_K | KVCR_CACHE_FUSED_FINALIZE)) return 0;
+  if ((flags & KVCR_CACHE_FP8_K) && (flags & KVCR_CACHE_FUSED_FINALIZE)) return 0;
   StorageLayout L;
   if (!make_layout(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
                    with_rope != 0, dtype == KVCR_BF16 ? 2 : 4, &L,
-                   (flags & KVCR_CACHE_FP8_K) != 0))
+                   (flags & KVCR_CACHE_FP8_K) != 0, (flags & KVCR_CACHE_FUSED_FINALIZE) != 0))
     return 0;
   return L.total;
 }
@@ -418,14 +446,21 @@ int kv_cache_init_ex(kvcr_cache** out, int sinks, int window, int aux_frames,
   if (dtype != KVCR_BF16 && dtype != KVCR_F32) return fail(KVCR_EINVAL, "kv_cache_init: bad dtype");
   if (head_dim != 64 && head_dim != 128)
     return fail(KVCR_EUNSUPPORTED, "kv_cache_init: head_dim must be 64 or 128");
-  if (flags & ~(unsigned)KVCR_CACHE_FP8_K) return fail(KVCR_EINVAL, "kv_cache_init: unknown flags");
+  if (flags & ~(unsigned)(KVCR_CACHE_FP8_K | KVCR_CACHE_FUSED_FINALIZE))
+    return fail(KVCR_EINVAL, "kv_cache_init: unknown flags");
   const bool fp8 = (flags & KVCR_CACHE_FP8_K) != 0;
+  const bool fused = (flags & KVCR_CACHE_FUSED_FINALIZE) != 0;
+  if (fp8 && fused)
+    return fail(KVCR_EINVAL, "kv_cache_init: KVCR_CACHE_FP8_K and KVCR_CACHE_FUSED_FINALIZE "
+                             "cannot be combined");
   if (fp8 && (dtype != KVCR_BF16 || head_dim != 128))
     return fail(KVCR_EUNSUPPORTED, "kv_cache_init: e4m3 K copies need bf16 and head_dim 128");
+  if (fused && dtype != KVCR_BF16)
+    return fail(KVCR_EUNSUPPORTED, "kv_cache_init: fused finalize needs bf16");
   if (sinks < 0 || window < 0 || aux_frames < 0 || sinks + window < 1 ||
-      sinks + window + aux_frames > kMaxSlots)
-    return fail(KVCR_ESHAPE,
-                "kv_cache_init: need 1 <= sinks + window and sinks + window + aux_frames <= 32");
+      sinks + window + aux_frames + (fused ? chunk_frames : 0) > kMaxSlots)
+    return fail(KVCR_ESHAPE, "kv_cache_init: need 1 <= sinks + window and sinks + window + "
+                             "aux_frames (+ chunk_frames spare slots) <= 32");
   if (tokens_per_frame < 1 || heads < 1 || chunk_frames < 1 || chunk_frames > kMaxFrames)
     return fail(KVCR_ESHAPE, "kv_cache_init: bad tokens_per_frame / heads / chunk_frames (<= 16)");
   if ((long long)chunk_frames * tokens_per_frame > (1LL << 30) ||
@@ -444,7 +479,7 @@ int kv_cache_init_ex(kvcr_cache** out, int sinks, int window, int aux_frames,
   const size_t esize = dtype == KVCR_BF16 ? 2 : 4;
   StorageLayout L;
   if (!make_layout(sinks, window, aux_frames, tokens_per_frame, heads, head_dim, chunk_frames,
-                   rope != nullptr, esize, &L, fp8))
+                   rope != nullptr, esize, &L, fp8, fused))
     return fail(KVCR_ESHAPE, "kv_cache_init: bad sizes");
   const bool has_storage = device_storage != nullptr;
   if (!has_storage && storage_bytes != 0)
@@ -479,6 +514,11 @@ int kv_cache_init_ex(kvcr_cache** out, int sinks, int window, int aux_frames,
   c->n_sm = n_sm;
   c->cc_major = cc;
   c->fp8 = fp8;
+  c->fused = fused;
+  c->phys.resize(sinks + window);
+  for (int i = 0; i < sinks + window; ++i) c->phys[i] = i;
+  if (fused)
+    for (int f = 0; f < chunk_frames; ++f) c->spare.push_back(sinks + window + aux_frames + f);
   c->slot_frame.assign(sinks + window, -1);
   c->n_sinks_filled = 0;
   c->last_frame = -1;
@@ -509,7 +549,8 @@ int kv_cache_init_ex(kvcr_cache** out, int sinks, int window, int aux_frames,
     }
     if (dtype == KVCR_BF16) {
       const uint64_t dims[4] = {(uint64_t)head_dim, (uint64_t)heads, (uint64_t)tokens_per_frame,
-                                (uint64_t)(sinks + window + aux_frames)};
+                                (uint64_t)(sinks + window + aux_frames +
+                                           (fused ? chunk_frames : 0))};
       int rc = encode_bf16_map(&c->tm_kc, c->storage + L.k_off, 4, dims, kKeyTile);
       if (!rc) rc = encode_bf16_map(&c->tm_vc, c->storage + L.v_off, 4, dims, kKeyTile);
       if (!rc && fp8) rc = encode_map(&c->tm_kc8, true, c->storage + L.k8_off, 4, dims, kKeyTile);
@@ -565,7 +606,7 @@ int kv_cache_append_rope(kvcr_cache* c, const void* k, const void* v, const int3
     for (int i = 0; i < n_frames; ++i) {
       // skip frames not retained, or evicted again by a later frame of this call
       if (slots[i] < 0 || c->slot_frame[slots[i]] != frame_idx[i]) continue;
-      p.dst_frame_off[n] = (long long)slots[i] * frame_elems;
+      p.dst_frame_off[n] = (long long)phys_of(c, slots[i]) * frame_elems;
       p.src_frame[n] = i;
       written.push_back(frame_idx[i]);
       written_slots.push_back(slots[i]);
@@ -674,8 +715,8 @@ int kv_cache_append_rope_batch(kvcr_cache* const* caches, int n_caches, const vo
         }
         p->src_a[n] = static_cast<const uint8_t*>(k[i]) + (size_t)f * frame_bytes;
         p->src_b[n] = static_cast<const uint8_t*>(v[i]) + (size_t)f * frame_bytes;
-        p->dst_a[n] = c->storage + c->lay.k_off + (size_t)slots[i][f] * frame_bytes;
-        p->dst_b[n] = c->storage + c->lay.v_off + (size_t)slots[i][f] * frame_bytes;
+        p->dst_a[n] = c->storage + c->lay.k_off + (size_t)phys_of(c, slots[i][f]) * frame_bytes;
+        p->dst_b[n] = c->storage + c->lay.v_off + (size_t)phys_of(c, slots[i][f]) * frame_bytes;
         p->tframe[n] = f;
         ++n;
       }
@@ -758,8 +799,9 @@ int kv_cache_slot_data(const kvcr_cache* c, int slot, const void** k, const void
   if (slot < 0 || slot >= c->S + c->W + c->A)
     return fail(KVCR_EINVAL, "kv_cache_slot_data: bad slot");
   const size_t frame = (size_t)c->T * c->H * c->D * c->esize;
-  *k = c->storage + c->lay.k_off + (size_t)slot * frame;
-  *v = c->storage + c->lay.v_off + (size_t)slot * frame;
+  const int ph = phys_of(c, slot);
+  *k = c->storage + c->lay.k_off + (size_t)ph * frame;
+  *v = c->storage + c->lay.v_off + (size_t)ph * frame;
   return KVCR_OK;
 }
 
@@ -771,9 +813,10 @@ int kv_cache_slot_data_fp8(const kvcr_cache* c, int slot, const void** k_codes,
     return fail(KVCR_ESTATE, "kv_cache_slot_data_fp8: the cache keeps no e4m3 K copies");
   if (slot < 0 || slot >= c->S + c->W + c->A)
     return fail(KVCR_EINVAL, "kv_cache_slot_data_fp8: bad slot");
-  *k_codes = c->storage + c->lay.k8_off + (size_t)slot * c->T * c->H * c->D;
+  const int ph = phys_of(c, slot);
+  *k_codes = c->storage + c->lay.k8_off + (size_t)ph * c->T * c->H * c->D;
   *k_scales = reinterpret_cast<const float*>(c->storage + c->lay.k8s_off) +
-              (size_t)slot * blocks_of(c->T) * c->H;
+              (size_t)ph * blocks_of(c->T) * c->H;
   return KVCR_OK;
 }
 
@@ -859,10 +902,7 @@ int chunk_attention_fwd(kvcr_cache* c, const void* q, int n_q, const void* k_cur
 
   // visible cached frames, in slot order
   int slots[kMaxSlots];
-  int n_vis = 0;
-  for (int i = 0; i < c->S + c->W; ++i)
-    if (c->slot_frame[i] >= 0) slots[n_vis++] = i;
-  for (int i = 0; i < c->n_aux; ++i) slots[n_vis++] = c->S + c->W + i;  // auxiliary frames
+  const int n_vis = visible_slots(c, slots);
 
   const void* q_src = q;
   const void* k_src = k_cur;
@@ -951,6 +991,131 @@ int chunk_attention_fwd(kvcr_cache* c, const void* q, int n_q, const void* k_cur
   return KVCR_OK;
 }
 
+// ====================================== chunk attention + finalize in one pass
+// The chunk's rotated K and its V go once into spare physical slots (one rope
+// copy launch), the queries are rotated into the scratch, the attention reads
+// the chunk's keys from the spare slots (as cached-frame tiles), and the append
+// is done by relabelling: each retained frame's anchor / window slot points at
+// the spare slot holding it, and the physical slot it replaced becomes spare.
+int chunk_attention_fwd_finalize(kvcr_cache* c, const void* q, int n_q, const void* k_cur,
+                                 const void* v_cur, const int32_t* cur_frame_idx,
+                                 int n_cur_frames, float softmax_scale, void* o, float* lse,
+                                 void* stream) {
+  const char* fn = "chunk_attention_fwd_finalize";
+  if (c == nullptr) return fail(KVCR_EINVAL, std::string(fn) + ": cache is NULL");
+  if (!c->has_storage) return fail(KVCR_ESTATE, std::string(fn) + ": bookkeeping-only cache");
+  if (!c->fused)
+    return fail(KVCR_ESTATE, std::string(fn) + ": the cache has no spare slots "
+                                               "(create it with KVCR_CACHE_FUSED_FINALIZE)");
+  if (n_cur_frames < 1 || n_cur_frames > c->F)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_cur_frames must be in [1, chunk_frames]");
+  if (n_q < 0) return fail(KVCR_ESHAPE, std::string(fn) + ": n_q < 0");
+  const int n_cur = n_cur_frames * c->T;
+  if (c->rope && n_q != n_cur)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": with RoPE n_q must be n_cur_frames * T");
+  int rc = check_frames(c, cur_frame_idx, n_cur_frames, fn);
+  if (rc) return rc;
+  if (!k_cur || !v_cur || (n_q > 0 && (!q || !o)))
+    return fail(KVCR_EINVAL, std::string(fn) + ": NULL tensor");
+  if (!aligned16(k_cur) || !aligned16(v_cur) || (n_q > 0 && (!aligned16(q) || !aligned16(o))))
+    return fail(KVCR_EINVAL, std::string(fn) + ": tensors must be 16-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(KVCR_EINVAL, std::string(fn) + ": lse must be 4-byte aligned");
+  if ((long long)n_q * c->H * c->D > (1LL << 31) - 1)
+    return fail(KVCR_ESHAPE, std::string(fn) + ": n_q too large");
+  if ((int)c->spare.size() < n_cur_frames)
+    return fail(KVCR_ESTATE, std::string(fn) + ": not enough spare slots");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)c->D);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // keys of this call: the visible cached / auxiliary frames, then the chunk's
+  // own frames from the spare slots they are written to
+  int slots[kMaxSlots];
+  int n_vis = visible_slots(c, slots);
+  for (int f = 0; f < n_cur_frames; ++f) slots[n_vis++] = c->spare[f];
+  const long long frame_elems = (long long)c->T * c->H * c->D;
+  cudaError_t e;
+  {  // rotated K and V of the chunk into the spare slots
+    RopeCopyParams p;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(c, p);
+    p.src_a = k_cur;
+    p.src_b = v_cur;
+    p.dst_a = c->storage + c->lay.k_off;
+    p.dst_b = c->storage + c->lay.v_off;
+    p.rotate_a = c->rope ? 1 : 0;
+    p.rotate_b = 0;
+    p.n_frames = n_cur_frames;
+    for (int f = 0; f < n_cur_frames; ++f) {
+      p.dst_frame_off[f] = (long long)c->spare[f] * frame_elems;
+      p.src_frame[f] = f;
+    }
+    if (c->rope) fill_ttab(c, p, cur_frame_idx, n_cur_frames);
+    LaunchScope scope(KVCR_K_APPEND_ROPE, s);
+    e = launch_rope_copy(p, c->dtype, s, c->n_sm);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd_finalize: write launch");
+  const void* q_src = q;
+  if (c->rope && n_q > 0) {  // rotated queries into the scratch
+    RopeCopyParams p;
+    std::memset(&p, 0, sizeof(p));
+    fill_common(c, p);
+    p.src_a = q;
+    p.dst_a = c->storage + c->lay.q_off;
+    p.rotate_a = 1;
+    p.n_frames = n_cur_frames;
+    for (int f = 0; f < n_cur_frames; ++f) {
+      p.dst_frame_off[f] = f * frame_elems;
+      p.src_frame[f] = f;
+    }
+    fill_ttab(c, p, cur_frame_idx, n_cur_frames);
+    LaunchScope scope(KVCR_K_ROPE_STAGE, s);
+    e = launch_rope_copy(p, c->dtype, s, c->n_sm);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd_finalize: stage launch");
+    q_src = c->storage + c->lay.q_off;
+  }
+  if (n_q > 0) {
+    ChunkAttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t dq[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_q};
+    const uint64_t dn[3] = {(uint64_t)c->D, (uint64_t)c->H, (uint64_t)n_cur};
+    rc = encode_bf16_map(&p.tm_q, q_src, 3, dq, kTile);
+    // no current-chunk tiles are read; the maps stay valid for the prefetch
+    if (!rc) rc = encode_bf16_map(&p.tm_kn, k_cur, 3, dn, kKeyTile);
+    if (!rc) rc = encode_bf16_map(&p.tm_vn, v_cur, 3, dn, kKeyTile);
+    if (rc) return rc;
+    p.tm_kc = c->tm_kc;
+    p.tm_vc = c->tm_vc;
+    p.c.o = o;
+    p.c.lse = lse;
+    p.c.n_q = n_q;
+    p.c.H = c->H;
+    p.c.scale_log2 = (float)(scale * 1.4426950408889634);
+    p.c.inject = inject_state().kind;
+    p.c.wait_ns = inject_state().wait_ns;
+    p.s.T = c->T;
+    p.s.n_vis = n_vis;
+    p.s.tiles_per_slot = (c->T + kKeyTile - 1) / kKeyTile;
+    p.s.n_cur = 0;
+    p.s.cur_tiles = 0;
+    for (int i = 0; i < n_vis; ++i) p.s.slots[i] = slots[i];
+    LaunchScope scope(KVCR_K_CHUNK_ATTN, s);
+    e = launch_chunk_attn_sm100(p, c->D, (n_q + kTile - 1) / kTile, s);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_fwd_finalize: attention launch");
+  }
+
+  // the append, by relabelling
+  std::vector<int> placed(n_cur_frames), evicted;
+  for (int i = 0; i < n_cur_frames; ++i) {
+    placed[i] = place_frame(c, cur_frame_idx[i], evicted);
+    if (placed[i] >= 0) std::swap(c->phys[placed[i]], c->spare[i]);
+  }
+  c->last_slots = placed;
+  c->last_evicted = evicted;
+  c->n_aux = 0;
+  return KVCR_OK;
+}
+
 // ============================================== chunk attention, e4m3 QK^T
 // Stage (RoPE) as chunk_attention_fwd(), quantize the staged queries and current
 // keys to e4m3 blocks of 128 tokens, then the tensor-core kernel with the QK^T
@@ -987,10 +1152,7 @@ int chunk_attention_fwd_fp8(kvcr_cache* c, const void* q, int n_q, const void* k
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   int slots[kMaxSlots];
-  int n_vis = 0;
-  for (int i = 0; i < c->S + c->W; ++i)
-    if (c->slot_frame[i] >= 0) slots[n_vis++] = i;
-  for (int i = 0; i < c->n_aux; ++i) slots[n_vis++] = c->S + c->W + i;  // auxiliary frames
+  const int n_vis = visible_slots(c, slots);
 
   const void* q_src = q;
   const void* k_src = k_cur;
@@ -1117,10 +1279,7 @@ int chunk_attention_fwd_static_scratch(kvcr_cache* c, const void* q, int n_q, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   int slots[kMaxSlots];
-  int n_vis = 0;
-  for (int i = 0; i < c->S + c->W; ++i)
-    if (c->slot_frame[i] >= 0) slots[n_vis++] = i;
-  for (int i = 0; i < c->n_aux; ++i) slots[n_vis++] = c->S + c->W + i;  // auxiliary frames
+  const int n_vis = visible_slots(c, slots);
 
   const void* q_src = q;
   const void* k_src = k_cur;

@@ -21,7 +21,8 @@ constexpr long long kWaitTimeoutNs = 2000000000LL;  // bounded device waits: 2 s
 // ------------------------------------------------------- rope / copy pass --
 // One launch moves n_frames frames of two tensors (a and b) of shape
 // [T][H][D] each from contiguous sources to per-frame destinations, rotating
-// a (and b when rotate_b) with the 3D rotary embedding.
+// a (and b when rotate_b) with the 3D rotary embedding.  src_b = NULL moves a
+// alone (single-cache kernel).
 struct RopeCopyParams {
   const void* src_a;
   const void* src_b;

@@ -165,6 +165,7 @@ __global__ void __launch_bounds__(256) rope_copy_kernel(const __grid_constant__ 
   const int pair0 = (lane % kVecPerRow) * kPairsPerVec;
   const long long tok_elems = (long long)p.H * D;
   const Elem* src_a = static_cast<const Elem*>(p.src_a) + (long long)p.src_frame[f] * p.T * tok_elems;
+  const bool has_b = p.src_b != nullptr;             // tensor b is optional
   const Elem* src_b = static_cast<const Elem*>(p.src_b) + (long long)p.src_frame[f] * p.T * tok_elems;
   Elem* dst_a = static_cast<Elem*>(p.dst_a) + p.dst_frame_off[f];
   Elem* dst_b = static_cast<Elem*>(p.dst_b) + p.dst_frame_off[f];
@@ -203,18 +204,21 @@ __global__ void __launch_bounds__(256) rope_copy_kernel(const __grid_constant__ 
         if (k0 + k < n_mine) {
           const long long off = base + (long long)(lane + 32 * (k0 + k)) * kPerVec;
           a[k] = ld_stream(src_a + off);
-          b[k] = ld_stream(src_b + off);
+          if (has_b) b[k] = ld_stream(src_b + off);
         }
       }
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) {
         if (k0 + k < n_mine) {
           const long long off = base + (long long)(lane + 32 * (k0 + k)) * kPerVec;
-          uint4 ra = a[k], rb = b[k];
+          uint4 ra = a[k];
           if (p.rotate_a) ra = rotate_vec<kPairsPerVec>(ra, cs);
-          if (p.rotate_b) rb = rotate_vec<kPairsPerVec>(rb, cs);
           st_vec(dst_a + off, ra);
-          st_vec(dst_b + off, rb);
+          if (has_b) {
+            uint4 rb = b[k];
+            if (p.rotate_b) rb = rotate_vec<kPairsPerVec>(rb, cs);
+            st_vec(dst_b + off, rb);
+          }
         }
       }
     }

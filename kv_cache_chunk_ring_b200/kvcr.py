@@ -21,7 +21,7 @@ KVCR_OK, KVCR_EINVAL, KVCR_ESHAPE, KVCR_ESTATE = 0, -1, -2, -3
 KVCR_ECUDA, KVCR_ETIMEOUT, KVCR_ESTORAGE, KVCR_EUNSUPPORTED = -4, -5, -6, -7
 KVCR_BF16, KVCR_F32 = 0, 1
 KVCR_TILE_EMPTY, KVCR_TILE_PARTIAL, KVCR_TILE_FULL = 0, 1, 2
-KVCR_CACHE_FP8_K = 1
+KVCR_CACHE_FP8_K, KVCR_CACHE_FUSED_FINALIZE = 1, 2
 (KVCR_K_APPEND_ROPE, KVCR_K_ROPE_STAGE, KVCR_K_CHUNK_ATTN, KVCR_K_MOBA_ATTN,
  KVCR_K_ATTN_F32, KVCR_K_MOBA_BWD_PREP, KVCR_K_MOBA_BWD_DKDV, KVCR_K_MOBA_BWD_DQ,
  KVCR_K_SET_AUX, KVCR_K_APPEND_BATCH, KVCR_K_QUANT_E4M3, KVCR_K_CHUNK_ATTN_FP8) = range(12)
@@ -36,7 +36,7 @@ KERNEL_NAMES = {KVCR_K_APPEND_ROPE: "append_rope", KVCR_K_ROPE_STAGE: "rope_stag
 EXPORTS = [
     "kv_cache_storage_bytes", "kv_cache_init", "kv_cache_storage_bytes_aux", "kv_cache_init_aux",
     "kv_cache_storage_bytes_ex", "kv_cache_init_ex", "kv_cache_slot_data_fp8",
-    "chunk_attention_fwd_fp8",
+    "chunk_attention_fwd_fp8", "chunk_attention_fwd_finalize",
     "kv_cache_set_aux", "kv_cache_num_aux", "kv_cache_append_rope", "kv_cache_append_rope_batch",
     "kv_cache_evict",
     "kv_cache_slot_map", "kv_cache_last_append", "kv_cache_num_cached", "kv_cache_slot_data",
@@ -180,6 +180,8 @@ def lib() -> ctypes.CDLL:
         "kv_cache_slot_data_fp8": (c_int, [c_p, c_int, ctypes.POINTER(c_p), ctypes.POINTER(c_p)]),
         "chunk_attention_fwd_fp8": (c_int, [c_p, c_p, c_int, c_p, c_p, i32p, c_int, c_f, c_p, c_p,
                                             c_p]),
+        "chunk_attention_fwd_finalize": (c_int, [c_p, c_p, c_int, c_p, c_p, i32p, c_int, c_f, c_p,
+                                                 c_p, c_p]),
         "kv_cache_set_aux": (c_int, [c_p, c_p, c_p, i32p, c_int, c_p]),
         "kv_cache_num_aux": (c_int, [c_p, ctypes.POINTER(c_int)]),
         "kv_cache_append_rope": (c_int, [c_p, c_p, c_p, i32p, c_int, c_p]),
@@ -423,6 +425,17 @@ def chunk_attention_fwd_fp8(handle, q, k_cur, v_cur, cur_frame_idx: Sequence[int
                                          _stream(stream)))
 
 
+def chunk_attention_fwd_finalize(handle, q, k_cur, v_cur, cur_frame_idx: Sequence[int], o,
+                                 lse=None, softmax_scale: float = 0.0, stream=None) -> None:
+    """chunk_attention_fwd then the append of k_cur, v_cur, in one pass over K and V (cache
+    made with KVCR_CACHE_FUSED_FINALIZE)."""
+    _check_chunk_args(handle, q, k_cur, v_cur, len(cur_frame_idx), o, lse)
+    _check(lib().chunk_attention_fwd_finalize(handle, _ptr(q), q.shape[0], _ptr(k_cur),
+                                              _ptr(v_cur), _i32(cur_frame_idx),
+                                              len(cur_frame_idx), float(softmax_scale), _ptr(o),
+                                              _ptr(lse), _stream(stream)))
+
+
 def kv_cache_slot_data_fp8(handle, slot: int) -> Tuple[int, int]:
     """Device addresses (ints) of one slot's e4m3 K codes and block scales."""
     k = ctypes.c_void_p()
@@ -527,9 +540,11 @@ class Cache:
 
     def __init__(self, sinks: int, window: int, tokens_per_frame: int, heads: int, head_dim: int,
                  chunk_frames: int, rope=None, dtype="bf16", device="cuda",
-                 bookkeeping_only: bool = False, aux_frames: int = 0, fp8_k: bool = False):
+                 bookkeeping_only: bool = False, aux_frames: int = 0, fp8_k: bool = False,
+                 fused_finalize: bool = False):
         self.sinks, self.window, self.aux_frames = sinks, window, aux_frames
-        self.flags = KVCR_CACHE_FP8_K if fp8_k else 0
+        self.flags = ((KVCR_CACHE_FP8_K if fp8_k else 0) |
+                      (KVCR_CACHE_FUSED_FINALIZE if fused_finalize else 0))
         self.T, self.H, self.D, self.F = tokens_per_frame, heads, head_dim, chunk_frames
         self.rope = rope
         self.dtype_code = _dtype_code(dtype)
@@ -608,6 +623,20 @@ class Cache:
             lse = torch.empty((self.H, q.shape[0]), dtype=torch.float32, device=q.device)
         fn = chunk_attention_fwd_fp8 if fp8 else chunk_attention_fwd
         fn(self.handle, q, k_cur, v_cur, frames, o, lse, softmax_scale, stream)
+        return o, lse
+
+    def attention_finalize(self, q, k_cur, v_cur, frames: Sequence[int], want_lse: bool = False,
+                           out=None, softmax_scale: float = 0.0, stream=None):
+        """The chunk's last step: attention, then k_cur, v_cur appended (one pass; cache
+        made with fused_finalize).  Returns (o, lse); the append's slots and evictions are
+        read with kv_cache_last_append."""
+        import torch
+        o = out if out is not None else torch.empty_like(q)
+        lse = None
+        if want_lse:
+            lse = torch.empty((self.H, q.shape[0]), dtype=torch.float32, device=q.device)
+        chunk_attention_fwd_finalize(self.handle, q, k_cur, v_cur, frames, o, lse, softmax_scale,
+                                     stream)
         return o, lse
 
     def slot_tensors_fp8(self, slot: int):

@@ -50,18 +50,19 @@ def rope_of(spec):
 
 def gpu_rollout(spec, chunks, rows_for: Optional[Callable] = None, use_rope: bool = True,
                 window_schedule: Optional[List[int]] = None, aux_for: Optional[Callable] = None,
-                aux_frames: int = 0):
+                aux_frames: int = 0, finalize: bool = False):
     """Run the rollout through the C ABI.  Returns dict of per-call outputs (rows
     selected by rows_for, numpy fp64), LSEs, slot maps after each append, and the
     Cache (for read-back).  ``aux_for(chunk)`` -> None or (k, v, positions) sets the
     chunk's auxiliary frames before its first step (cache built with
-    ``aux_frames`` auxiliary slots)."""
+    ``aux_frames`` auxiliary slots).  ``finalize``: each chunk's last step is one
+    chunk_attention_fwd_finalize call (attention and append in one pass)."""
     import torch
-    from kv_cache_chunk_ring_b200.kvcr import Cache
+    from kv_cache_chunk_ring_b200.kvcr import Cache, kv_cache_last_append
     cap = spec.window if window_schedule is None else max(spec.window, max(window_schedule))
     cache = Cache(spec.sinks, cap, spec.tokens_per_frame, spec.heads, spec.head_dim,
                   spec.chunk_frames, rope=spec.rope() if use_rope else None, dtype=spec.dtype,
-                  aux_frames=aux_frames)
+                  aux_frames=aux_frames, fused_finalize=finalize)
     out = dict(outputs=[], lses=[], slot_maps=[], appended=[], cache=cache)
     for item in chunks:
         c, s, frames = item["chunk"], item["step"], item["frames"]
@@ -74,13 +75,20 @@ def gpu_rollout(spec, chunks, rows_for: Optional[Callable] = None, use_rope: boo
         q = to_dev(item["q"], spec.dtype)
         k = to_dev(item["k"], spec.dtype)
         v = to_dev(item["v"], spec.dtype)
-        o, lse = cache.attention(q, k, v, frames, want_lse=True)
+        last = s == spec.steps - 1
+        if finalize and last:
+            o, lse = cache.attention_finalize(q, k, v, frames, want_lse=True)
+        else:
+            o, lse = cache.attention(q, k, v, frames, want_lse=True)
         rows = np.arange(q.shape[0]) if rows_for is None else np.asarray(rows_for(c, s))
         idx = torch.from_numpy(rows).cuda()
         out["outputs"].append(to_np(o.index_select(0, idx)))
         out["lses"].append(lse.index_select(1, idx).cpu().numpy().astype(np.float64))
-        if s == spec.steps - 1:
-            out["appended"].append(cache.append(k, v, frames))
+        if last:
+            if finalize:
+                out["appended"].append(kv_cache_last_append(cache.handle, len(frames)))
+            else:
+                out["appended"].append(cache.append(k, v, frames))
             out["slot_maps"].append(cache.slot_map())
     torch.cuda.synchronize()
     return out

@@ -269,3 +269,50 @@ def test_moba_longest_sequence_accepted_and_one_more_rejected():
     assert e.value.code == kvcr.KVCR_ESHAPE
     cls = kvcr.moba_classify_tiles(16, 16384, 0, 128)
     assert cls.shape == (4096, 4096)
+
+
+def test_cache_flags():
+    F, T, H = 2, 12, 2
+    base = kvcr.kv_cache_storage_bytes_ex(2, 3, 0, T, H, 128, F, 1, kvcr.KVCR_BF16, 0)
+    fused = kvcr.kv_cache_storage_bytes_ex(2, 3, 0, T, H, 128, F, 1, kvcr.KVCR_BF16,
+                                           kvcr.KVCR_CACHE_FUSED_FINALIZE)
+    # two spare frame slots of K and V (bf16), each 256-byte aligned
+    assert fused - base >= 2 * F * T * H * 128 * 2
+    assert fused - base < 2 * F * T * H * 128 * 2 + 2 * 256
+    fp8 = kvcr.kv_cache_storage_bytes_ex(2, 3, 0, T, H, 128, F, 1, kvcr.KVCR_BF16,
+                                         kvcr.KVCR_CACHE_FP8_K)
+    # e4m3 K of 5 slots + their scales + two chunks of e4m3 staging (and scales)
+    assert fp8 - base >= 5 * T * H * 128 + 2 * F * T * H * 128
+    both = kvcr.KVCR_CACHE_FP8_K | kvcr.KVCR_CACHE_FUSED_FINALIZE
+    assert kvcr.kv_cache_storage_bytes_ex(2, 3, 0, T, H, 128, F, 1, kvcr.KVCR_BF16, both) == 0
+    assert kvcr.kv_cache_storage_bytes_ex(2, 3, 0, T, H, 128, F, 1, kvcr.KVCR_BF16, 8) == 0
+    for flags, dtype, D, code in [(both, kvcr.KVCR_BF16, 128, kvcr.KVCR_EINVAL),
+                                  (8, kvcr.KVCR_BF16, 128, kvcr.KVCR_EINVAL),
+                                  (kvcr.KVCR_CACHE_FP8_K, kvcr.KVCR_BF16, 64,
+                                   kvcr.KVCR_EUNSUPPORTED),
+                                  (kvcr.KVCR_CACHE_FP8_K, kvcr.KVCR_F32, 128,
+                                   kvcr.KVCR_EUNSUPPORTED),
+                                  (kvcr.KVCR_CACHE_FUSED_FINALIZE, kvcr.KVCR_F32, 64,
+                                   kvcr.KVCR_EUNSUPPORTED)]:
+        with pytest.raises(kvcr.KvcrError) as e:
+            kvcr.kv_cache_init_ex(2, 3, 0, T, H, D, F, None, dtype, flags, None)
+        assert e.value.code == code, (flags, dtype, D)
+    # spare slots count against the 32 frame slots
+    with pytest.raises(kvcr.KvcrError) as e:
+        kvcr.kv_cache_init_ex(6, 20, 4, T, H, 128, 4, None, kvcr.KVCR_BF16,
+                              kvcr.KVCR_CACHE_FUSED_FINALIZE, None)
+    assert e.value.code == kvcr.KVCR_ESHAPE
+    h = kvcr.kv_cache_init_ex(6, 20, 2, T, H, 128, 4, None, kvcr.KVCR_BF16,
+                              kvcr.KVCR_CACHE_FUSED_FINALIZE, None)
+    kvcr.kv_cache_destroy(h)
+
+
+def test_new_entry_points_need_their_cache_kind():
+    """Bookkeeping-only caches refuse attention; the e4m3 and fused entry points also
+    refuse a cache made without their flag (before any launch)."""
+    h = kvcr.kv_cache_init(1, 2, 4, 1, 128, 1, None, kvcr.KVCR_BF16, None)
+    L = kvcr.lib()
+    for fn in (L.chunk_attention_fwd_fp8, L.chunk_attention_fwd_finalize):
+        rc = fn(h, None, 4, None, None, kvcr._i32([3]), 1, 0.0, None, None, None)
+        assert rc == kvcr.KVCR_ESTATE
+    kvcr.kv_cache_destroy(h)
