@@ -397,7 +397,9 @@ int moba_classify_tiles(const kvcr_moba_layout *layout, int tile, uint8_t *cls, 
 
 /* Synchronise `stream` and return (then clear) the device-side status of the
  * library's kernels on the current device: KVCR_OK or KVCR_ETIMEOUT when a
- * kernel gave up on a bounded wait (its outputs are then invalid).  Library
+ * kernel gave up on a bounded wait (its outputs are then invalid; the forward
+ * attention kernels write NaN into the rows and LSE of a query tile that gave
+ * up, so a missed check still shows in the output).  Library
  * convention (failure detection); no page has a counterpart. */
 int kvcr_check_status(void *stream);
 

@@ -654,8 +654,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     if (ok && n_tiles > 0) ok = wait_bar(&ctl->o_done[tq], 0, ctl);
     ok = __all_sync(0xFFFFFFFFu, ok);
     tc_fence_after();
-    const bool row_ok = ok && row_g < p.c.n_q;
-    const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+    // a CTA that gave up on a wait writes NaN rows (and NaN LSE): its outputs are
+    // invalid, and a caller that missed kvcr_check_status() still sees it
+    const bool row_ok = row_g < p.c.n_q;
+    const float inv_l = !ok ? __int_as_float(0x7FC00000) : (l_sum > 0.f ? 1.f / l_sum : 0.f);
     __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.c.o) + ((size_t)row_g * p.c.H + h) * HD;
 #pragma unroll 1
     for (int c = 0; c < HD / 32; ++c) {
@@ -682,7 +684,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
     }
     if (row_ok && p.c.lse != nullptr) {
-      const float lse = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+      const float lse = !ok ? __int_as_float(0x7FC00000)
+                            : (l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.6931471805599453f
+                                           : -INFINITY);
       p.c.lse[(size_t)h * p.c.n_q + row_g] = lse;
     }
   }

@@ -40,6 +40,8 @@ def test_withheld_signal_times_out_and_context_survives():
         with pytest.raises(kvcr.KvcrError) as e:
             kvcr.kvcr_check_status()
         assert e.value.code == kvcr.KVCR_ETIMEOUT
+        # every CTA gave up (each withholds one signal): its rows are NaN, not stale data
+        assert torch.isnan(o_bad.float()).all()
     finally:
         kvcr.kvcr_debug_inject(0, 0)
 
