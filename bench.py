@@ -217,7 +217,7 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
     T, H, D, F = spec.tokens_per_frame, h1 - h0, spec.head_dim, spec.chunk_frames
     stream = torch.cuda.current_stream()
 
-    cache = kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope())
+    cache = kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope(), fused_finalize=True)
     # seeded synthetic chunks: fill chunks + a pool for timing, this rank's heads
     gen = wl.rollout_chunks(wl.shrink(spec, n_chunks=STEADY_CHUNK + POOL), layer=layer)
     chunks = []
@@ -276,6 +276,27 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
         if n:
             kt[name] = {"launches": n, "avg_ms": ms / n}
     kvcr.kvcr_trace_reset()
+
+    # ---------------- the same step as one fused call (attention + append) ----------------
+    def step_fused(i):
+        q, k, v = chunks[STEADY_CHUNK + (i % POOL)]
+        frames = list(range(frame[0], frame[0] + F))
+        cache.attention_finalize(q, k, v, frames, out=o)
+        frame[0] += F
+
+    for i in range(args.warmup):
+        step_fused(i)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(args.steps):
+        step_fused(i)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    fused_ms = max_over_ranks(f0.elapsed_time(f1), dist, dev)
 
     # ---------------- end to end through the public API with host buffers ----------------
     # Every step uploads its Q, K, V from pinned host memory and downloads its O.  Two
@@ -366,6 +387,9 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
         "kernels": {k: {"launches": v["launches"], "avg_ms": round(v["avg_ms"], 5)}
                     for k, v in kt.items()},
         "attn_ms_per_call": round(attn_ms + kt.get("rope_stage", {}).get("avg_ms", 0.0), 5),
+        "ms_per_step_fused_call": round(fused_ms / args.steps, 4),
+        "value_fused_call": round(whole_job_throughput(job_ranks, args.steps, step_flops(spec),
+                                                       fused_ms), 2),
         "attn_kernel_pct_of_peak": round(100 * achieved / peak, 2),
         "append_gb_s": round(app_gbs, 1),
         "append_hbm_frac": round(app_gbs / float(peaks["hbm_gbs"]), 4),
@@ -521,8 +545,10 @@ def run_layers30(args, clocks=False) -> dict:
     _build.build()
     spec = wl.VIDEO_832x464_30L
     T, H, D, F = spec.tokens_per_frame, spec.heads, spec.head_dim, spec.chunk_frames
-    caches = [kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope())
-              for _ in range(spec.layers)]
+    # spare slots for the fused last step (chunk_attention_fwd_finalize); the other
+    # paths use these caches like plain ones
+    caches = [kvcr.Cache(spec.sinks, spec.window, T, H, D, F, rope=spec.rope(),
+                         fused_finalize=True) for _ in range(spec.layers)]
     gen = torch.Generator(device="cuda").manual_seed(spec.seed)
     pool = [tuple(_randn((spec.chunk_tokens, H, D), gen) for _ in range(3)) for _ in range(6)]
     o = torch.empty_like(pool[0][0])
@@ -553,6 +579,19 @@ def run_layers30(args, clocks=False) -> dict:
         kvcr.append_batch(caches, ks, vs, frames)
         frame[0] += F
 
+    def chunk_fused():
+        # the same chunk with each layer's last step attending and appending in one call
+        frames = list(range(frame[0], frame[0] + F))
+        for li, c in enumerate(caches):
+            for s in range(spec.steps):
+                q, k, v = pool[n_call[0] % len(pool)]
+                n_call[0] += 1
+                if s == spec.steps - 1:
+                    c.attention_finalize(q, k, v, frames, out=o)
+                else:
+                    c.attention(q, k, v, frames, out=o)
+        frame[0] += F
+
     for _ in range(STEADY_CHUNK):
         chunk()
     kvcr.kvcr_trace_reset()
@@ -561,6 +600,7 @@ def run_layers30(args, clocks=False) -> dict:
         sampler.start()
     ms = _timed(chunk, args.steps, args.warmup)
     ms_batched = _timed(chunk_batched, args.steps, args.warmup)
+    ms_fused = _timed(chunk_fused, args.steps, args.warmup)
     clk = sampler.stop() if sampler else None
     kvcr.kvcr_trace_enable(True)
     chunk()
@@ -586,6 +626,7 @@ def run_layers30(args, clocks=False) -> dict:
             "append_kernel_us": round(1e3 * app_ms / max(1, app_n), 2),
             "append_gb_s": round(append_bytes(spec) / (app_ms / max(1, app_n) * 1e-3) / 1e9, 1),
             "ms_per_chunk_batched_append": round(ms_batched, 3),
+            "ms_per_chunk_fused_last_step": round(ms_fused, 3),
             "append_batch_kernel_us": round(1e3 * bat_ms / max(1, bat_n), 2),
             "append_batch_gb_s": round(spec.layers * append_bytes(spec) /
                                        (bat_ms / max(1, bat_n) * 1e-3) / 1e9, 1),
@@ -929,6 +970,7 @@ def main():
                 out.update({
                     "layers30_ms_per_chunk": l30["ms_per_chunk_batched_append"],
                     "layers30_ms_per_chunk_separate_appends": l30["ms_per_chunk"],
+                    "layers30_ms_per_chunk_fused_last_step": l30["ms_per_chunk_fused_last_step"],
                     "layers30_attn_kernel_ms": l30["attn_kernel_ms"],
                     "layers30_attn_kernel_frac": l30["attn_kernel_frac"],
                     "layers30_append_gb_s": l30["append_batch_gb_s"],

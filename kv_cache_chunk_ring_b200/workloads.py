@@ -35,10 +35,11 @@ def round_to_bf16(x: np.ndarray) -> np.ndarray:
     inputs (the inputs here are finite normal draws).
     """
     x = np.ascontiguousarray(x, dtype=np.float32)
-    bits = x.view(np.uint32).astype(np.uint64)
-    lsb = (bits >> 16) & 1
-    rounded = ((bits + 0x7FFF + lsb) >> 16) << 16
-    return rounded.astype(np.uint32).view(np.float32)
+    bits = x.view(np.uint32)
+    lsb = (bits >> np.uint32(16)) & np.uint32(1)
+    # finite inputs stay below 2^32 after the addition (largest: 0xFF7FFFFF + 0x8000)
+    rounded = (bits + np.uint32(0x7FFF) + lsb) & np.uint32(0xFFFF0000)
+    return rounded.view(np.float32)
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:

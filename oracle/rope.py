@@ -71,18 +71,18 @@ def rope3d(x: np.ndarray, t: np.ndarray, h: np.ndarray, w: np.ndarray,
         raise ValueError("pairs must cover head_dim")
     pos = (np.asarray(t, dtype=np.float64), np.asarray(h, dtype=np.float64),
            np.asarray(w, dtype=np.float64))
-    out = x.copy()
+    # angle of every (token, pair): pair i of axis a (index j in it) turns by pos_a * freq
+    ang = np.empty((N, D // 2))
     for i in range(D // 2):
         axis, j = axis_of_pair(i, pairs)
-        p_axis = pairs[axis]
-        freq = base ** (-(2.0 * j) / (2.0 * p_axis))
-        ang = pos[axis] * freq                      # [N]
-        c = np.cos(ang)[:, None]
-        s = np.sin(ang)[:, None]
-        x0 = x[:, :, 2 * i]
-        x1 = x[:, :, 2 * i + 1]
-        out[:, :, 2 * i] = x0 * c - x1 * s
-        out[:, :, 2 * i + 1] = x0 * s + x1 * c
+        ang[:, i] = pos[axis] * base ** (-(2.0 * j) / (2.0 * pairs[axis]))
+    c = np.cos(ang)[:, None, :]                      # [N, 1, D/2]
+    s = np.sin(ang)[:, None, :]
+    x0 = x[:, :, 0::2]                               # first element of each pair
+    x1 = x[:, :, 1::2]
+    out = np.empty_like(x)
+    out[:, :, 0::2] = x0 * c - x1 * s
+    out[:, :, 1::2] = x0 * s + x1 * c
     return out
 
 

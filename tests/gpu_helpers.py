@@ -44,6 +44,60 @@ def assert_close(got, ref, what: str = "", max_abs=TOL_MAX_ABS, rel_rms=TOL_REL_
     return ma, rr
 
 
+def tee(items, maxsize: int = 2):
+    """Two iterators over one pass of ``items`` (each item produced once), for an oracle
+    rollout running in a thread beside the GPU rollout; at most ``maxsize`` items wait
+    in either queue, so memory stays bounded."""
+    import queue
+    import threading
+    end = object()
+    qs = (queue.Queue(maxsize), queue.Queue(maxsize))
+
+    def produce():
+        for x in items:
+            for q in qs:
+                q.put(x)
+        for q in qs:
+            q.put(end)
+
+    threading.Thread(target=produce, daemon=True).start()
+
+    def drain(q):
+        while True:
+            x = q.get()
+            if x is end:
+                return
+            yield x
+    return drain(qs[0]), drain(qs[1])
+
+
+def oracle_and_gpu(items, oracle_fn, gpu_fn):
+    """Run ``oracle_fn(iterator)`` in a thread and ``gpu_fn(iterator)`` here over one pass of
+    ``items``; returns (oracle result, gpu result)."""
+    import threading
+    a, b = tee(items)
+    box = {}
+
+    def run():
+        try:
+            box["ref"] = oracle_fn(a)
+        except BaseException as e:  # re-raised below
+            box["err"] = e
+            for _ in a:             # keep the producer from blocking
+                pass
+    th = threading.Thread(target=run)
+    th.start()
+    try:
+        got = gpu_fn(b)
+    finally:
+        for _ in b:
+            pass
+        th.join()
+    if "err" in box:
+        raise box["err"]
+    return box["ref"], got
+
+
 def rope_of(spec):
     return spec.rope()
 

@@ -9,7 +9,8 @@ from kv_cache_chunk_ring_b200 import workloads as wl
 from oracle.attn import attention
 from oracle.rollout import rollout
 from oracle.rope import rope3d, rope_positions
-from tests.gpu_helpers import (TOL_LSE, assert_close, gpu_rollout, to_dev, to_np, errors)
+from tests.gpu_helpers import (TOL_LSE, assert_close, gpu_rollout, oracle_and_gpu, to_dev, to_np,
+                               errors)
 
 pytestmark = pytest.mark.gpu
 
@@ -89,8 +90,9 @@ def test_832x464_rollout_40_chunks():
             return np.arange(L)
         return wl.sample_rows(L, 1024, 1000 + c, list(range(128)) + list(range(L - 16, L)))
 
-    ref = rollout(spec, wl.rollout_chunks(spec), rows_for=rows_for)
-    got = gpu_rollout(spec, wl.rollout_chunks(spec), rows_for=rows_for)
+    ref, got = oracle_and_gpu(wl.rollout_chunks(spec),
+                              lambda it: rollout(spec, it, rows_for=rows_for),
+                              lambda it: gpu_rollout(spec, it, rows_for=rows_for))
     assert len(got["outputs"]) == spec.n_chunks
     worst = (0.0, 0.0)
     for n, (o, o_ref, l, l_ref) in enumerate(zip(got["outputs"], ref.outputs, got["lses"],

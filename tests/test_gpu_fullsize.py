@@ -14,7 +14,7 @@ from kv_cache_chunk_ring_b200 import workloads as wl
 from oracle.attn import attention
 from oracle.moba import MobaLayout, moba_attention_rows
 from oracle.rollout import rollout
-from tests.gpu_helpers import TOL_LSE, assert_close, gpu_rollout, to_dev, to_np
+from tests.gpu_helpers import TOL_LSE, assert_close, gpu_rollout, oracle_and_gpu, to_dev, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -51,8 +51,9 @@ def test_30layer_rollout_layer(layer):
     def rows_for(c, s):
         return _rows(L, 48, 5000 + 100 * layer + 10 * c + s)
 
-    ref = rollout(spec, wl.rollout_chunks(spec, layer), rows_for=rows_for)
-    got = gpu_rollout(spec, wl.rollout_chunks(spec, layer), rows_for=rows_for)
+    ref, got = oracle_and_gpu(wl.rollout_chunks(spec, layer),
+                              lambda it: rollout(spec, it, rows_for=rows_for),
+                              lambda it: gpu_rollout(spec, it, rows_for=rows_for))
     assert len(got["outputs"]) == spec.n_chunks * spec.steps
     worst = _check(ref, got, f"layer {layer}")
     print(f"30-layer rollout layer {layer}: worst max_abs={worst[0]:.3e} rel_rms={worst[1]:.3e}")
@@ -71,8 +72,10 @@ def test_720p_dynamic_window_and_cross_attention():
     def rows_for(c, s):
         return _rows(L, 256, 7000 + c)
 
-    ref = rollout(spec, wl.rollout_chunks(spec), rows_for=rows_for, window_schedule=sched)
-    got = gpu_rollout(spec, wl.rollout_chunks(spec), rows_for=rows_for, window_schedule=sched)
+    ref, got = oracle_and_gpu(
+        wl.rollout_chunks(spec),
+        lambda it: rollout(spec, it, rows_for=rows_for, window_schedule=sched),
+        lambda it: gpu_rollout(spec, it, rows_for=rows_for, window_schedule=sched))
     assert len(got["outputs"]) == spec.n_chunks == 60
     worst = _check(ref, got, "720p dynamic window")
     assert [a[0] for a in got["appended"]] == ref.appended_slots

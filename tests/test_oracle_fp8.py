@@ -204,3 +204,16 @@ def test_fp8_rollout_error_against_exact_is_a_few_percent():
     for a, b in zip(exact.outputs, low.outputs):
         rel = np.linalg.norm(a - b) / np.linalg.norm(a)
         assert 1e-3 < rel < 8e-2, rel
+
+
+def test_input_draws_round_to_bf16_like_torch():
+    """The seeded inputs are N(0, 1) float32 draws rounded to bf16 (nearest, ties to even);
+    the shared generator's rounding agrees with torch's conversion, ties included."""
+    torch = pytest.importorskip("torch")
+    from kv_cache_chunk_ring_b200 import workloads as wl
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(200000).astype(np.float32) * np.float32(3.0)
+    ties = (np.arange(1, 2000, dtype=np.uint32) << 16 | np.uint32(0x8000)).view(np.float32)
+    x = np.concatenate([x, ties, -ties])
+    ref = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(wl.round_to_bf16(x), ref)
