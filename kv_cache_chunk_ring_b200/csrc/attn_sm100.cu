@@ -66,8 +66,12 @@ constexpr float kRescaleLog2 = 8.0f;
 // P of a tile is released to the MMA in this many parts of 128 / kPParts keys.
 constexpr int kPParts = 2;
 // Of the 16 key pairs in each 32-key group, pairs [0, kExpSfuPairs) take exp2 on
-// the SFU and the rest on the FMA pipe.
+// the SFU and the rest on the FMA pipe.  With bf16 QK^T all go to the SFU; with
+// the e4m3 QK^T (half the S product time) moving 2 of 16 pairs to the FMA pipe
+// measured 4-5 % faster (0.78 against 0.81-0.82 ms per 832x464 call), while the
+// same split slowed the bf16 kernel by about 1 %.
 constexpr int kExpSfuPairs = 16;
+constexpr int kExpSfuPairsE4m3 = 14;
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S_t / P_t at t * 128, O_t at 256 + t * 128.
 constexpr uint32_t kTmemS = 0;
@@ -619,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                                         __uint_as_float(s[32 * c + 2 * e + 1]));
           const float2 x = ffma2(sv, sl2x2, negm);
           float2 pv;
-          if (e >= kExpSfuPairs) {                   // this share of the exps on the FMA pipe
+          if (e >= (kFp8 ? kExpSfuPairsE4m3 : kExpSfuPairs)) {  // this share on the FMA pipe
             pv = ex2_fma2(x);
           } else {
             pv = make_float2(ex2_sfu(x.x), ex2_sfu(x.y));
