@@ -258,6 +258,19 @@ int kv_cache_slot_data_fp8(const kvcr_cache *c, int slot, const void **k_codes,
  * Slots sinks + window .. + aux_frames - 1 are the auxiliary slots. */
 int kv_cache_slot_data(const kvcr_cache *c, int slot, const void **k, const void **v);
 
+/* Checkpoint of a cache's host state: the slot table, the anchors filled, the window's
+ * recency order, the last frame index, the physical relabelling of a fused-finalize
+ * cache, the auxiliary count and the last append's record.  Together with a copy of
+ * the caller-owned device storage it restores a cache after a restart without
+ * replaying its appends (library convention; the pages describe the state, not a
+ * format).  Export: *size receives the byte count; buf = NULL only queries it;
+ * KVCR_ESTORAGE when cap < *size.  Import into a cache created with the same
+ * configuration (sizes, dtype, RoPE, flags): KVCR_ESHAPE for another configuration,
+ * KVCR_EINVAL for a truncated or inconsistent state; nothing changes on error.  The
+ * format is little-endian int32 words headed by "KVCR" and a version.  Host only. */
+int kv_cache_export_state(const kvcr_cache *c, void *buf, size_t cap, size_t *size);
+int kv_cache_import_state(kvcr_cache *c, const void *buf, size_t size);
+
 void kv_cache_destroy(kvcr_cache *c);
 
 /* ------------------------------------------------------------ attention --- */

@@ -870,6 +870,160 @@ int kv_cache_set_aux(kvcr_cache* c, const void* k, const void* v, const int32_t*
   return KVCR_OK;
 }
 
+// ==================================================== host state checkpoint
+// Layout (int32 words): magic, version, then the configuration (S, W, A, T, H, D, F,
+// dtype, rope, grid_h, grid_w, pairs_t, pairs_h, pairs_w, base as two words, fp8,
+// fused), then the state: slot_frame[S + W], n_sinks_filled, last_frame, n_aux,
+// phys[S + W], n_spare, spare[], n_recent, recent[], n_last_slots, last_slots[],
+// n_last_evicted, last_evicted[].
+namespace {
+constexpr int32_t kStateMagic = 0x5243564B;  // "KVCR"
+constexpr int32_t kStateVersion = 1;
+
+void config_words(const kvcr_cache* c, std::vector<int32_t>& w) {
+  int32_t base[2];
+  std::memcpy(base, &c->rp.base, sizeof(double));
+  const int32_t cfg[] = {c->S, c->W, c->A, c->T, c->H, c->D, c->F, (int32_t)c->dtype,
+                         c->rope ? 1 : 0, c->rope ? c->rp.grid_h : 0, c->rope ? c->rp.grid_w : 0,
+                         c->rope ? c->rp.pairs_t : 0, c->rope ? c->rp.pairs_h : 0,
+                         c->rope ? c->rp.pairs_w : 0, c->rope ? base[0] : 0,
+                         c->rope ? base[1] : 0, c->fp8 ? 1 : 0, c->fused ? 1 : 0};
+  w.insert(w.end(), std::begin(cfg), std::end(cfg));
+}
+
+void state_words(const kvcr_cache* c, std::vector<int32_t>& w) {
+  w.push_back(kStateMagic);
+  w.push_back(kStateVersion);
+  config_words(c, w);
+  w.insert(w.end(), c->slot_frame.begin(), c->slot_frame.end());
+  w.push_back(c->n_sinks_filled);
+  w.push_back(c->last_frame);
+  w.push_back(c->n_aux);
+  w.insert(w.end(), c->phys.begin(), c->phys.end());
+  w.push_back((int32_t)c->spare.size());
+  w.insert(w.end(), c->spare.begin(), c->spare.end());
+  w.push_back((int32_t)c->recent.size());
+  w.insert(w.end(), c->recent.begin(), c->recent.end());
+  w.push_back((int32_t)c->last_slots.size());
+  w.insert(w.end(), c->last_slots.begin(), c->last_slots.end());
+  w.push_back((int32_t)c->last_evicted.size());
+  w.insert(w.end(), c->last_evicted.begin(), c->last_evicted.end());
+}
+}  // namespace
+
+int kv_cache_export_state(const kvcr_cache* c, void* buf, size_t cap, size_t* size) {
+  if (c == nullptr || size == nullptr) return fail(KVCR_EINVAL, "kv_cache_export_state: NULL");
+  std::vector<int32_t> w;
+  state_words(c, w);
+  *size = w.size() * sizeof(int32_t);
+  if (buf == nullptr) return KVCR_OK;
+  if (cap < *size) return fail(KVCR_ESTORAGE, "kv_cache_export_state: buffer too small");
+  std::memcpy(buf, w.data(), *size);
+  return KVCR_OK;
+}
+
+int kv_cache_import_state(kvcr_cache* c, const void* buf, size_t size) {
+  const char* fn = "kv_cache_import_state";
+  if (c == nullptr || buf == nullptr) return fail(KVCR_EINVAL, std::string(fn) + ": NULL");
+  if (size % sizeof(int32_t) != 0) return fail(KVCR_EINVAL, std::string(fn) + ": truncated");
+  const size_t n = size / sizeof(int32_t);
+  std::vector<int32_t> w(n);
+  std::memcpy(w.data(), buf, size);
+  size_t at = 0;
+  bool short_buf = false;
+  auto next = [&]() -> int32_t {
+    if (at >= n) {
+      short_buf = true;
+      return 0;
+    }
+    return w[at++];
+  };
+  auto bad = [&](const char* why) { return fail(KVCR_EINVAL, std::string(fn) + ": " + why); };
+  if (next() != kStateMagic || next() != kStateVersion)
+    return bad("not a cache state of this version");
+  std::vector<int32_t> cfg_want;
+  config_words(c, cfg_want);
+  for (int32_t v : cfg_want)
+    if (next() != v || short_buf)
+      return fail(KVCR_ESHAPE, std::string(fn) + ": the state belongs to a cache of another "
+                                                 "configuration");
+  const int SW = c->S + c->W;
+  std::vector<int> slot_frame(SW), phys(SW), spare, recent_v, last_slots, last_evicted;
+  for (int i = 0; i < SW; ++i) slot_frame[i] = next();
+  const int n_sinks_filled = next();
+  const int last_frame = next();
+  const int n_aux = next();
+  for (int i = 0; i < SW; ++i) phys[i] = next();
+  auto read_list = [&](std::vector<int>& out, int limit) -> bool {
+    const int k = next();
+    if (short_buf || k < 0 || k > limit) return false;
+    out.resize(k);
+    for (int i = 0; i < k; ++i) out[i] = next();
+    return !short_buf;
+  };
+  if (!read_list(spare, kMaxSlots) || !read_list(recent_v, c->W) ||
+      !read_list(last_slots, kMaxFrames) || !read_list(last_evicted, kMaxSlots + kMaxFrames))
+    return bad("malformed lists");
+  if (short_buf || at != n) return bad("wrong length");
+  // consistency of the slot table
+  if (n_sinks_filled < 0 || n_sinks_filled > c->S) return bad("anchor count out of range");
+  if (n_aux < 0 || n_aux > c->A) return bad("auxiliary count out of range");
+  int max_cached = -1;
+  std::vector<int> cached;
+  for (int i = 0; i < SW; ++i) {
+    const int f = slot_frame[i];
+    if (f < -1) return bad("negative frame");
+    if (i < c->S && ((i < n_sinks_filled) != (f >= 0))) return bad("anchor slots inconsistent");
+    if (f >= 0) {
+      cached.push_back(f);
+      max_cached = std::max(max_cached, f);
+    }
+  }
+  std::sort(cached.begin(), cached.end());
+  if (std::adjacent_find(cached.begin(), cached.end()) != cached.end())
+    return bad("a frame is cached twice");
+  if (last_frame < max_cached) return bad("last frame below a cached frame");
+  for (size_t i = 0; i < recent_v.size(); ++i) {
+    if (i > 0 && recent_v[i] <= recent_v[i - 1]) return bad("window frames not increasing");
+    int hits = 0;
+    for (int s = c->S; s < SW; ++s) hits += slot_frame[s] == recent_v[i];
+    if (hits != 1) return bad("window frame not in exactly one window slot");
+  }
+  int window_used = 0;
+  for (int s = c->S; s < SW; ++s) window_used += slot_frame[s] >= 0;
+  if (window_used != (int)recent_v.size()) return bad("window slots and recency list differ");
+  // the physical relabelling: a permutation of the non-auxiliary frame slots
+  const int n_phys = SW + c->A + (c->fused ? c->F : 0);
+  std::vector<int> seen(n_phys, 0);
+  if ((int)spare.size() != (c->fused ? c->F : 0)) return bad("spare slot count");
+  for (int v : phys) {
+    if (v < 0 || v >= n_phys || (v >= SW && v < SW + c->A)) return bad("physical slot range");
+    seen[v]++;
+  }
+  for (int v : spare) {
+    if (v < 0 || v >= n_phys || (v >= SW && v < SW + c->A)) return bad("spare slot range");
+    seen[v]++;
+  }
+  for (int v = 0; v < n_phys; ++v)
+    if ((v >= SW && v < SW + c->A) ? seen[v] != 0 : seen[v] != 1)
+      return bad("physical slots are not a permutation");
+  for (int v : last_slots)
+    if (v < -1 || v >= SW) return bad("appended slot out of range");
+  for (int v : last_evicted)
+    if (v < 0) return bad("negative evicted frame");
+  // commit
+  c->slot_frame = slot_frame;
+  c->n_sinks_filled = n_sinks_filled;
+  c->last_frame = last_frame;
+  c->n_aux = n_aux;
+  c->phys = phys;
+  c->spare = spare;
+  c->recent.assign(recent_v.begin(), recent_v.end());
+  c->last_slots = last_slots;
+  c->last_evicted = last_evicted;
+  return KVCR_OK;
+}
+
 int kv_cache_num_aux(const kvcr_cache* c, int* n) {
   if (c == nullptr || n == nullptr) return fail(KVCR_EINVAL, "kv_cache_num_aux: NULL");
   *n = c->n_aux;

@@ -36,7 +36,8 @@ KERNEL_NAMES = {KVCR_K_APPEND_ROPE: "append_rope", KVCR_K_ROPE_STAGE: "rope_stag
 EXPORTS = [
     "kv_cache_storage_bytes", "kv_cache_init", "kv_cache_storage_bytes_aux", "kv_cache_init_aux",
     "kv_cache_storage_bytes_ex", "kv_cache_init_ex", "kv_cache_slot_data_fp8",
-    "chunk_attention_fwd_fp8", "chunk_attention_fwd_finalize",
+    "chunk_attention_fwd_fp8", "chunk_attention_fwd_finalize", "kv_cache_export_state",
+    "kv_cache_import_state",
     "kv_cache_set_aux", "kv_cache_num_aux", "kv_cache_append_rope", "kv_cache_append_rope_batch",
     "kv_cache_evict",
     "kv_cache_slot_map", "kv_cache_last_append", "kv_cache_num_cached", "kv_cache_slot_data",
@@ -178,6 +179,8 @@ def lib() -> ctypes.CDLL:
                                      c_int, ctypes.POINTER(kvcr_rope), c_int, ctypes.c_uint, c_p,
                                      c_sz]),
         "kv_cache_slot_data_fp8": (c_int, [c_p, c_int, ctypes.POINTER(c_p), ctypes.POINTER(c_p)]),
+        "kv_cache_export_state": (c_int, [c_p, c_p, c_sz, ctypes.POINTER(c_sz)]),
+        "kv_cache_import_state": (c_int, [c_p, c_p, c_sz]),
         "chunk_attention_fwd_fp8": (c_int, [c_p, c_p, c_int, c_p, c_p, i32p, c_int, c_f, c_p, c_p,
                                             c_p]),
         "chunk_attention_fwd_finalize": (c_int, [c_p, c_p, c_int, c_p, c_p, i32p, c_int, c_f, c_p,
@@ -402,6 +405,21 @@ def kv_cache_slot_data(handle, slot: int) -> Tuple[int, int]:
     return int(k.value), int(v.value)
 
 
+def kv_cache_export_state(handle) -> bytes:
+    """The cache's host state (slot table, recency, relabelling, counts) as bytes."""
+    n = ctypes.c_size_t()
+    _check(lib().kv_cache_export_state(handle, None, 0, ctypes.byref(n)))
+    buf = ctypes.create_string_buffer(n.value)
+    _check(lib().kv_cache_export_state(handle, buf, n.value, ctypes.byref(n)))
+    return buf.raw[:n.value]
+
+
+def kv_cache_import_state(handle, state: bytes) -> None:
+    """Restore a state from kv_cache_export_state into a cache of the same configuration."""
+    buf = ctypes.create_string_buffer(bytes(state), len(state))
+    _check(lib().kv_cache_import_state(handle, buf, len(state)))
+
+
 def kv_cache_destroy(handle) -> None:
     _CACHE_INFO.pop(handle.value if isinstance(handle, ctypes.c_void_p) else handle, None)
     lib().kv_cache_destroy(handle)
@@ -594,6 +612,13 @@ class Cache:
 
     def num_aux(self) -> int:
         return kv_cache_num_aux(self.handle)
+
+    def export_state(self) -> bytes:
+        """Host state for a checkpoint (save it with a copy of ``self.storage``)."""
+        return kv_cache_export_state(self.handle)
+
+    def import_state(self, state: bytes) -> None:
+        kv_cache_import_state(self.handle, state)
 
     def slot_map(self) -> List[int]:
         return kv_cache_slot_map(self.handle, self.sinks + self.window)
