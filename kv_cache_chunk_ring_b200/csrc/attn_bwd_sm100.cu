@@ -23,18 +23,23 @@
 //            dK  += dS^T Q_i             (TS: dS^T in TMEM, Q_i MN-major)  384-511
 //          Thread r of each warpgroup owns key r (TMEM lane r); warpgroup w
 //          handles query columns [64 w, 64 w + 64), so LSE and D are per column,
-//          staged per stage in shared memory (one 1 KB bulk copy).  P^T (bf16)
-//          overwrites S^T and dS^T overwrites dP^T in TMEM; MMAs of one thread
-//          run in issue order, so the next S^T / dP^T is issued right after the
-//          MMAs that read the current ones.
+//          staged per stage in shared memory (one 1 KB bulk copy).  Once a
+//          warpgroup has read its half of S^T and of dP^T into registers, it
+//          writes P^T (bf16 pairs) into the first 32 and dS^T into the last 32
+//          of its 64 dP^T columns.  The S^T columns are then free, so S^T(i+1)
+//          is issued as soon as they are read and stage i+1 has landed, ahead
+//          of dV_i when it can, and overlaps tile i's exponentials; dP^T(i+1)
+//          follows dK_i (MMAs of one thread run in issue order).
 //   dQ     one CTA per (head, 128-query tile), the key tiles it may read
 //          streaming through the ring:
 //            S  = Q K_j^T (SS, cols 0-127)   dP = dO V_j^T (SS, cols 128-255)
 //            dQ += dS K_j (TS: dS in TMEM, K_j MN-major; cols 256-383)
 //          Thread r owns query r; LSE and D are per row (registers).
-// Roles as in the forward kernel: warp 8 issues the TMA copies, one thread of
-// warp 9 the MMAs, warps 0-7 (two warpgroups, registers raised with setmaxnreg)
-// the elementwise work and the epilogue.  Every wait is bounded (2 s): a thread
+// Roles as in the forward kernel: warp 8 issues the TMA copies, warp 9 the MMAs
+// (one elected lane of the converged warp; elect.sync picks the same lane every
+// time, so its products run in issue order and its commits track them), warps
+// 0-7 (two warpgroups, registers raised with setmaxnreg) the elementwise work
+// and the epilogue.  Every wait is bounded (2 s): a thread
 // that gives up records KVCR_ETIMEOUT, raises the CTA abort flag, and the CTA
 // drains its copies and MMAs before freeing TMEM.
 #include <cuda_bf16.h>
@@ -126,7 +131,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, BwdCtl*
   return true;
 }
 
-// wait_bar for the MMA-issuing thread: non-suspending polls.
+// wait_bar for the MMA-issuing warp: non-suspending polls.
 __device__ __forceinline__ bool spin_bar(uint64_t* bar, uint32_t parity, BwdCtl* ctl) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -142,6 +147,26 @@ __device__ __forceinline__ bool spin_bar(uint64_t* bar, uint32_t parity, BwdCtl*
     }
   }
   return true;
+}
+
+// Time / abort check of a hand-written poll loop: true when the CTA is aborting or
+// the wait that began at t0 ran out (recording KVCR_ETIMEOUT and raising abort).
+__device__ __forceinline__ bool poll_expired(BwdCtl* ctl, uint64_t t0) {
+  if (*reinterpret_cast<volatile int*>(&ctl->abort)) return true;
+  if (globaltimer() - t0 > ctl->wait_ns) {
+    atomicExch(&g_bwd_status, (int)KVCR_ETIMEOUT);
+    *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+    return true;
+  }
+  return false;
+}
+
+// spin_bar for the whole MMA warp: every lane polls (a completed phase stays
+// completed until the warp's own later products let the next one finish), and the
+// lanes agree on the outcome before the warp goes on, converged.
+__device__ __forceinline__ bool spin_bar_w(uint64_t* bar, uint32_t parity, BwdCtl* ctl) {
+  const bool ok = spin_bar(bar, parity, ctl);
+  return __all_sync(0xFFFFFFFFu, ok);
 }
 
 // Wait used while draining after an abort: ignores the abort flag, bounded.
@@ -288,8 +313,8 @@ __device__ __forceinline__ void mma_ss_tiles(uint32_t d, uint32_t a, uint32_t b)
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
     const uint32_t off = (kk >> 2) * BwdSmem<HD>::kBoxBytes + (kk & 3) * 32;
-    umma_ss(d, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(b + off, 16, 1024), kIdesc,
-            kk > 0 ? 1u : 0u);
+    umma_ss_w(d, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(b + off, 16, 1024), kIdesc,
+              kk > 0 ? 1u : 0u);
   }
 }
 
@@ -302,9 +327,9 @@ __device__ __forceinline__ void mma_ts_half(uint32_t d, uint32_t a_base, uint32_
 #pragma unroll
   for (int k4 = 0; k4 < 4; ++k4) {
     const int kk = 4 * half + k4;
-    umma_ts(d, a_base + (uint32_t)(half * 64 + k4 * 8),
-            sdesc_sw128(b + kk * 16 * 128, BwdSmem<HD>::kBoxBytes, 1024), kIdesc,
-            (first && kk == 0) ? 0u : 1u);
+    umma_ts_w(d, a_base + (uint32_t)(half * 64 + k4 * 8),
+              sdesc_sw128(b + kk * 16 * 128, BwdSmem<HD>::kBoxBytes, 1024), kIdesc,
+              (first && kk == 0) ? 0u : 1u);
   }
 }
 
@@ -330,51 +355,75 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
     if (warp == kWarpTma) {
       if (lane == 0 && n_tiles > 0) bwd_producer<HD, true>(p, ctl, smem, h, kt);
     } else if (warp == kWarpMma) {
-      if (lane == 0 && n_tiles > 0) {
+      if (n_tiles > 0) {          // the whole warp: operands stay warp-uniform
         const uint32_t sK = smem_u32(smem + L::kA), sV = smem_u32(smem + L::kB);
         const uint32_t sQ = smem_u32(smem + L::kX), sDO = smem_u32(smem + L::kY);
-        bool ok = spin_bar(&ctl->fixed_full, 0, ctl) && spin_bar(&ctl->st_full[0], 0, ctl);
+        bool ok = spin_bar_w(&ctl->fixed_full, 0, ctl) && spin_bar_w(&ctl->st_full[0], 0, ctl);
         if (ok) {
           tc_fence_after();
           mma_ss_tiles<HD>(tmem + kTmemS, sK, sQ);      // S^T(0)
-          umma_commit(&ctl->s_full);
+          umma_commit_w(&ctl->s_full);
           mma_ss_tiles<HD>(tmem + kTmemDP, sV, sDO);    // dP^T(0)
-          umma_commit(&ctl->dp_full);
+          umma_commit_w(&ctl->dp_full);
         }
         for (int i = 0; ok && i < n_tiles; ++i) {
           const int st = i % kStages;
+          const int sn = (i + 1) % kStages;
           const bool more = i + 1 < n_tiles;
           const uint32_t ph = (uint32_t)i & 1u;
+          const uint32_t phn = (uint32_t)((i + 1) / kStages) & 1u;
+          // S^T(i+1) goes as soon as the softmax has read S^T(i) and stage i+1 has
+          // landed, ahead of dV_i if it can: P^T(i) lives in the dP^T columns, so
+          // the S^T columns are free once read, and the next S^T overlaps this
+          // tile's exponentials instead of following its dV.
+          bool s_pending = more;
           for (int w = 0; ok && w < 2; ++w) {           // dV += P^T dO_i
-            if (!(ok = spin_bar(&ctl->p_full[w], ph, ctl))) break;
+            const uint64_t t0 = globaltimer();
+            uint32_t n = 0;
+            for (;;) {
+              if (s_pending &&
+                  __all_sync(0xFFFFFFFFu, mbar_test_wait(&ctl->s_free, ph) &&
+                                              mbar_test_wait(&ctl->st_full[sn], phn))) {
+                tc_fence_after();
+                mma_ss_tiles<HD>(tmem + kTmemS, sK, sQ + sn * L::kTileBytes);   // S^T(i+1)
+                umma_commit_w(&ctl->s_full);
+                s_pending = false;
+              }
+              if (__all_sync(0xFFFFFFFFu, mbar_test_wait(&ctl->p_full[w], ph))) break;
+              if ((++n & 255u) == 0u && __any_sync(0xFFFFFFFFu, poll_expired(ctl, t0))) {
+                ok = false;
+                break;
+              }
+            }
+            if (!ok) break;
             tc_fence_after();
-            mma_ts_half<HD>(tmem + kTmemAcc0, tmem + kTmemS, sDO + st * L::kTileBytes, w, i == 0);
+            mma_ts_half<HD>(tmem + kTmemAcc0, tmem + kTmemDP, sDO + st * L::kTileBytes, w, i == 0);
           }
           if (!ok) break;
-          const int sn = (i + 1) % kStages;
-          if (more) {
-            if (!(ok = spin_bar(&ctl->st_full[sn], (uint32_t)((i + 1) / kStages) & 1u, ctl)))
+          if (s_pending) {
+            if (!(ok = spin_bar_w(&ctl->s_free, ph, ctl) && spin_bar_w(&ctl->st_full[sn], phn, ctl)))
               break;
             tc_fence_after();
             mma_ss_tiles<HD>(tmem + kTmemS, sK, sQ + sn * L::kTileBytes);   // S^T(i+1)
-            umma_commit(&ctl->s_full);
+            umma_commit_w(&ctl->s_full);
           }
           for (int w = 0; ok && w < 2; ++w) {           // dK += dS^T Q_i
-            if (!(ok = spin_bar(&ctl->ds_full[w], ph, ctl))) break;
+            if (!(ok = spin_bar_w(&ctl->ds_full[w], ph, ctl))) break;
             tc_fence_after();
-            mma_ts_half<HD>(tmem + kTmemAcc1, tmem + kTmemDP, sQ + st * L::kTileBytes, w, i == 0);
+            mma_ts_half<HD>(tmem + kTmemAcc1, tmem + kTmemDP + 32u, sQ + st * L::kTileBytes, w,
+                            i == 0);
           }
           if (!ok) break;
-          umma_commit(&ctl->st_empty[st]);
+          umma_commit_w(&ctl->st_empty[st]);
           if (more) {
             mma_ss_tiles<HD>(tmem + kTmemDP, sV, sDO + sn * L::kTileBytes);  // dP^T(i+1)
-            umma_commit(&ctl->dp_full);
+            umma_commit_w(&ctl->dp_full);
           } else {
-            umma_commit(&ctl->acc_done);
+            umma_commit_w(&ctl->acc_done);
           }
         }
         if (!ok) {
-          umma_commit(&ctl->drain);
+          umma_commit_w(&ctl->drain);
           drain_wait(&ctl->drain, 0);
         }
       }
@@ -408,6 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
       tmem_ld_32x32b_x32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_ld_32x32b_x32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
       tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&ctl->s_free);                    // S^T columns may take S^T(i+1)
       // lse * log2 e (l4) and D (d4) of columns 4m .. 4m + 3 of this warpgroup
       const float4* l4 = reinterpret_cast<const float4*>(smem + L::kW + st * kWsBytes) + wg * 16;
       const float4* d4 = l4 + kTile / 4;
@@ -422,28 +473,17 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
       float pr[64];
       const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t packed[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int n = 32 * c + 2 * q;
-          const float4 lv = l4[n >> 2];
-          const float2 x = ffma2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])),
-                                 sl2x2, (q & 1) ? make_float2(-lv.z, -lv.w)
-                                                : make_float2(-lv.x, -lv.y));
-          float p0 = ex2_sfu(x.x), p1 = ex2_sfu(x.y);
-          if (!((keep[c] >> (2 * q)) & 1u)) p0 = 0.f;
-          if (!((keep[c] >> (2 * q + 1)) & 1u)) p1 = 0.f;
-          pr[n] = p0;
-          pr[n + 1] = p1;
-          packed[q] = pack_bf16(p0, p1);
-        }
-        tmem_st_32x32b_x16(s_addr + c * 16, packed);
+      for (int n = 0; n < 64; n += 2) {
+        const float4 lv = l4[n >> 2];
+        const float2 x = ffma2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])),
+                               sl2x2, (n & 2) ? make_float2(-lv.z, -lv.w)
+                                              : make_float2(-lv.x, -lv.y));
+        float p0 = ex2_sfu(x.x), p1 = ex2_sfu(x.y);
+        if (!((keep[n >> 5] >> (n & 31)) & 1u)) p0 = 0.f;
+        if (!((keep[n >> 5] >> ((n + 1) & 31)) & 1u)) p1 = 0.f;
+        pr[n] = p0;
+        pr[n + 1] = p1;
       }
-      tmem_st_wait();
-      tc_fence_before();
-      // test hook: warpgroup 1 withholds its first P-ready arrival
-      if (!(p.inject == 1 && wg == 1 && i == 0)) mbar_arrive(&ctl->p_full[wg]);
 
       ok = wait_bar(&ctl->dp_full, (uint32_t)i & 1u, ctl);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
@@ -454,6 +494,19 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
       tmem_ld_32x32b_x32(dp_addr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_ld_32x32b_x32(dp_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
       tmem_ld_wait();
+      // This warpgroup's dP^T half is in registers now: P^T (bf16 pairs) takes
+      // its first 32 columns, dS^T its last 32.
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t packed[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) packed[q] = pack_bf16(pr[32 * c + 2 * q], pr[32 * c + 2 * q + 1]);
+        tmem_st_32x32b_x16(dp_addr + c * 16, packed);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      // test hook: warpgroup 1 withholds its first P-ready arrival
+      if (!(p.inject == 1 && wg == 1 && i == 0)) mbar_arrive(&ctl->p_full[wg]);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t packed[16];
@@ -465,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
           const float d1 = pr[n + 1] * (__uint_as_float(s[n + 1]) - ((q & 1) ? dv.w : dv.y));
           packed[q] = pack_bf16(d0, d1);
         }
-        tmem_st_32x32b_x16(dp_addr + c * 16, packed);
+        tmem_st_32x32b_x16(dp_addr + 32 + c * 16, packed);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -537,46 +590,46 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
     if (warp == kWarpTma) {
       if (lane == 0 && n_tiles > 0) bwd_producer<HD, false>(p, ctl, smem, h, qt);
     } else if (warp == kWarpMma) {
-      if (lane == 0 && n_tiles > 0) {
+      if (n_tiles > 0) {          // the whole warp: operands stay warp-uniform
         const uint32_t sQ = smem_u32(smem + L::kA), sDO = smem_u32(smem + L::kB);
         const uint32_t sK = smem_u32(smem + L::kX), sV = smem_u32(smem + L::kY);
-        bool ok = spin_bar(&ctl->fixed_full, 0, ctl) && spin_bar(&ctl->st_full[0], 0, ctl);
+        bool ok = spin_bar_w(&ctl->fixed_full, 0, ctl) && spin_bar_w(&ctl->st_full[0], 0, ctl);
         if (ok) {
           tc_fence_after();
           mma_ss_tiles<HD>(tmem + kTmemS, sQ, sK);      // S(0)
-          umma_commit(&ctl->s_full);
+          umma_commit_w(&ctl->s_full);
           mma_ss_tiles<HD>(tmem + kTmemDP, sDO, sV);    // dP(0)
-          umma_commit(&ctl->dp_full);
+          umma_commit_w(&ctl->dp_full);
         }
         for (int j = 0; ok && j < n_tiles; ++j) {
           const int st = j % kStages;
           const bool more = j + 1 < n_tiles;
           const uint32_t ph = (uint32_t)j & 1u;
           const int sn = (j + 1) % kStages;
-          if (!(ok = spin_bar(&ctl->s_free, ph, ctl))) break;
+          if (!(ok = spin_bar_w(&ctl->s_free, ph, ctl))) break;
           if (more) {
-            if (!(ok = spin_bar(&ctl->st_full[sn], (uint32_t)((j + 1) / kStages) & 1u, ctl)))
+            if (!(ok = spin_bar_w(&ctl->st_full[sn], (uint32_t)((j + 1) / kStages) & 1u, ctl)))
               break;
             tc_fence_after();
             mma_ss_tiles<HD>(tmem + kTmemS, sQ, sK + sn * L::kTileBytes);   // S(j+1)
-            umma_commit(&ctl->s_full);
+            umma_commit_w(&ctl->s_full);
           }
           for (int w = 0; ok && w < 2; ++w) {           // dQ += dS K_j
-            if (!(ok = spin_bar(&ctl->ds_full[w], ph, ctl))) break;
+            if (!(ok = spin_bar_w(&ctl->ds_full[w], ph, ctl))) break;
             tc_fence_after();
             mma_ts_half<HD>(tmem + kTmemAcc0, tmem + kTmemDP, sK + st * L::kTileBytes, w, j == 0);
           }
           if (!ok) break;
-          umma_commit(&ctl->st_empty[st]);
+          umma_commit_w(&ctl->st_empty[st]);
           if (more) {
             mma_ss_tiles<HD>(tmem + kTmemDP, sDO, sV + sn * L::kTileBytes);  // dP(j+1)
-            umma_commit(&ctl->dp_full);
+            umma_commit_w(&ctl->dp_full);
           } else {
-            umma_commit(&ctl->acc_done);
+            umma_commit_w(&ctl->acc_done);
           }
         }
         if (!ok) {
-          umma_commit(&ctl->drain);
+          umma_commit_w(&ctl->drain);
           drain_wait(&ctl->drain, 0);
         }
       }
