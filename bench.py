@@ -116,7 +116,7 @@ def recorded_traffic(record="chunk_attn_832x464.json", names=ATTN_SOURCES):
 class ClockSampler:
     """nvidia-smi clock / throttle samples during the timed region."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -126,6 +126,12 @@ class ClockSampler:
         self.dev = ids[device_index] if device_index < len(ids) else str(device_index)
         self.proc = None
         self.path = os.path.join(tempfile.gettempdir(), f"kvcr_clocks_{os.getpid()}.csv")
+        self.t0 = self.t1 = None
+
+    def window(self, t0: float, t1: float):
+        """Wall-clock bounds (time.time()) of the timed region: only samples taken
+        inside it are summarised."""
+        self.t0, self.t1 = t0, t1
 
     def start(self):
         try:
@@ -133,7 +139,7 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "25"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -151,14 +157,20 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             cols = [c.strip() for c in line.split(",")]
-            if len(cols) < 9:
+            if len(cols) < 10:
                 continue
             try:
-                sm.append(float(cols[1]))
-                mx = float(cols[2])
+                stamp, frac = (cols[0].split(".") + ["0"])[:2]
+                t = time.mktime(time.strptime(stamp, "%Y/%m/%d %H:%M:%S")) + float("0." + frac)
+                clk = float(cols[2])
+                top = float(cols[3])
             except ValueError:
                 continue
-            for n, c in zip(names, cols[5:9]):
+            if self.t0 is not None and not (self.t0 <= t <= self.t1):
+                continue                      # outside the timed region
+            sm.append(clk)
+            mx = top
+            for n, c in zip(names, cols[6:10]):
                 if c.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
@@ -245,21 +257,24 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
     # ---------------- timed region (device events, no tracing) ----------------
     sampler = ClockSampler(dev.index)
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.5)                                   # nvidia-smi up and sampling
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = kvcr.kvcr_launch_count()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
     ev0.record(stream)
     for i in range(args.steps):
         step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
+    w1 = time.time()
     if dist is not None:
         dist.barrier()
     launches = kvcr.kvcr_launch_count() - launches0
+    sampler.window(w0, w1)
     clocks = sampler.stop()
     elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
 
@@ -378,7 +393,11 @@ def run_ours(args, rank: int, world: int, dist) -> dict:
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": recorded_traffic(),
                      "kernel": "chunk_attn (tcgen05 attention, one launch per step)",
-                     "peak_source": f"{peak_kind} bf16_tflops (burst)"},
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                     # the timed loop runs long enough to meet the 1 kW power cap; the
+                     # same achieved rate against the sustained (power-capped) figure:
+                     "frac_sustained": round(achieved / float(
+                         peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])), 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
                 "h2d_bytes_per_step": 3 * chunk_bytes, "d2h_bytes_per_step": chunk_bytes,
                 "ms_per_step": round(e2e_ms / args.steps, 4),
@@ -483,7 +502,7 @@ def cpu_baseline(budget_s: float = 15.0) -> dict:
 
 def run_reference(args) -> dict:
     """The oracle as the reference arm: each step = the bounded oracle sample."""
-    per_step_budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    per_step_budget = max(0.2, 150.0 / max(1, args.steps + args.warmup))  # ~150 s in all
     run, flops, n = oracle_sample(32)
     t0 = time.perf_counter()
     run()
@@ -601,9 +620,14 @@ def run_layers30(args, clocks=False) -> dict:
     sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
     if sampler:
         sampler.start()
+        time.sleep(0.5)                               # nvidia-smi up and sampling
+    w0 = time.time()
     ms = _timed(chunk, args.steps, args.warmup)
     ms_batched = _timed(chunk_batched, args.steps, args.warmup)
     ms_fused = _timed(chunk_fused, args.steps, args.warmup)
+    w1 = time.time()
+    if sampler:
+        sampler.window(w0, w1)
     clk = sampler.stop() if sampler else None
     kvcr.kvcr_trace_enable(True)
     chunk()
@@ -916,7 +940,7 @@ def run_fp8(args) -> dict:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
