@@ -75,7 +75,8 @@ constexpr int kWsBytes = kTile * 8;  // (lse, D) of one 128-row tile
 
 struct __align__(8) BwdCtl {
   uint64_t fixed_full;                         // the CTA's own two tiles
-  uint64_t st_full[kStages], st_empty[kStages];
+  uint64_t x_full[kStages];                    // stage: first streamed tile (Q_i or K_j)
+  uint64_t st_full[kStages], st_empty[kStages];  // the rest of the stage; the whole stage
   uint64_t s_full, dp_full, s_free;
   uint64_t p_full[2], ds_full[2];              // per warpgroup (column half)
   uint64_t acc_done;
@@ -238,6 +239,7 @@ __device__ __forceinline__ void bwd_setup(const MobaBwdParams& p, BwdCtl* ctl, i
   if (threadIdx.x == 0) {
     mbar_init(&ctl->fixed_full, 1);
     for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctl->x_full[s], 1);
       mbar_init(&ctl->st_full[s], 1);
       mbar_init(&ctl->st_empty[s], 1);
     }
@@ -283,7 +285,9 @@ __device__ void bwd_producer(const MobaBwdParams& p, BwdCtl* ctl, uint8_t* smem,
   mbar_arrive_expect_tx(&ctl->fixed_full, 2 * L::kTileBytes);
   load_tile<HD>(fa, smem + L::kA, &ctl->fixed_full, h, tile * kTile);
   load_tile<HD>(fb, smem + L::kB, &ctl->fixed_full, h, tile * kTile);
-  constexpr uint32_t kStageBytes = 2 * L::kTileBytes + (kByKey ? kWsBytes : 0);
+  // the first streamed tile (Q_i, K_j) is copied first and has a barrier of its
+  // own: the next S-type product needs only it, and starts before the rest lands
+  constexpr uint32_t kRestBytes = L::kTileBytes + (kByKey ? kWsBytes : 0);
   int issued = 0;
   bool ok = true;
   for (int i = 0; i < n_tiles; ++i) {
@@ -291,8 +295,9 @@ __device__ void bwd_producer(const MobaBwdParams& p, BwdCtl* ctl, uint8_t* smem,
     const uint32_t ph = (uint32_t)(i / kStages) & 1u;
     const int u = (int)(ctl->tiles[i] & 0xFFFu);
     if (!(ok = wait_bar(&ctl->st_empty[st], ph ^ 1u, ctl))) break;
-    mbar_arrive_expect_tx(&ctl->st_full[st], kStageBytes);
-    load_tile<HD>(sx, smem + L::kX + st * L::kTileBytes, &ctl->st_full[st], h, u * kTile);
+    mbar_arrive_expect_tx(&ctl->x_full[st], L::kTileBytes);
+    load_tile<HD>(sx, smem + L::kX + st * L::kTileBytes, &ctl->x_full[st], h, u * kTile);
+    mbar_arrive_expect_tx(&ctl->st_full[st], kRestBytes);
     load_tile<HD>(sy, smem + L::kY + st * L::kTileBytes, &ctl->st_full[st], h, u * kTile);
     if (kByKey)
       bulk_load(smem + L::kW + st * kWsBytes, p.ws + ((size_t)h * p.s.n_units + u) * 2 * kTile,
@@ -301,8 +306,10 @@ __device__ void bwd_producer(const MobaBwdParams& p, BwdCtl* ctl, uint8_t* smem,
   }
   if (!ok) {
     drain_wait(&ctl->fixed_full, 0);
-    for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
+    for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i) {
+      drain_wait(&ctl->x_full[i % kStages], (uint32_t)(i / kStages) & 1u);
       drain_wait(&ctl->st_full[i % kStages], (uint32_t)(i / kStages) & 1u);
+    }
   }
 }
 
@@ -358,11 +365,15 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
       if (n_tiles > 0) {          // the whole warp: operands stay warp-uniform
         const uint32_t sK = smem_u32(smem + L::kA), sV = smem_u32(smem + L::kB);
         const uint32_t sQ = smem_u32(smem + L::kX), sDO = smem_u32(smem + L::kY);
-        bool ok = spin_bar_w(&ctl->fixed_full, 0, ctl) && spin_bar_w(&ctl->st_full[0], 0, ctl);
+        bool ok = spin_bar_w(&ctl->fixed_full, 0, ctl) && spin_bar_w(&ctl->x_full[0], 0, ctl);
         if (ok) {
           tc_fence_after();
           mma_ss_tiles<HD>(tmem + kTmemS, sK, sQ);      // S^T(0)
           umma_commit_w(&ctl->s_full);
+          ok = spin_bar_w(&ctl->st_full[0], 0, ctl);
+        }
+        if (ok) {
+          tc_fence_after();
           mma_ss_tiles<HD>(tmem + kTmemDP, sV, sDO);    // dP^T(0)
           umma_commit_w(&ctl->dp_full);
         }
@@ -383,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
             for (;;) {
               if (s_pending &&
                   __all_sync(0xFFFFFFFFu, mbar_test_wait(&ctl->s_free, ph) &&
-                                              mbar_test_wait(&ctl->st_full[sn], phn))) {
+                                              mbar_test_wait(&ctl->x_full[sn], phn))) {
                 tc_fence_after();
                 mma_ss_tiles<HD>(tmem + kTmemS, sK, sQ + sn * L::kTileBytes);   // S^T(i+1)
                 umma_commit_w(&ctl->s_full);
@@ -401,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
           }
           if (!ok) break;
           if (s_pending) {
-            if (!(ok = spin_bar_w(&ctl->s_free, ph, ctl) && spin_bar_w(&ctl->st_full[sn], phn, ctl)))
+            if (!(ok = spin_bar_w(&ctl->s_free, ph, ctl) && spin_bar_w(&ctl->x_full[sn], phn, ctl)))
               break;
             tc_fence_after();
             mma_ss_tiles<HD>(tmem + kTmemS, sK, sQ + sn * L::kTileBytes);   // S^T(i+1)
@@ -416,6 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
           if (!ok) break;
           umma_commit_w(&ctl->st_empty[st]);
           if (more) {
+            if (!(ok = spin_bar_w(&ctl->st_full[sn], phn, ctl))) break;
+            tc_fence_after();
             mma_ss_tiles<HD>(tmem + kTmemDP, sV, sDO + sn * L::kTileBytes);  // dP^T(i+1)
             umma_commit_w(&ctl->dp_full);
           } else {
@@ -593,11 +606,15 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
       if (n_tiles > 0) {          // the whole warp: operands stay warp-uniform
         const uint32_t sQ = smem_u32(smem + L::kA), sDO = smem_u32(smem + L::kB);
         const uint32_t sK = smem_u32(smem + L::kX), sV = smem_u32(smem + L::kY);
-        bool ok = spin_bar_w(&ctl->fixed_full, 0, ctl) && spin_bar_w(&ctl->st_full[0], 0, ctl);
+        bool ok = spin_bar_w(&ctl->fixed_full, 0, ctl) && spin_bar_w(&ctl->x_full[0], 0, ctl);
         if (ok) {
           tc_fence_after();
           mma_ss_tiles<HD>(tmem + kTmemS, sQ, sK);      // S(0)
           umma_commit_w(&ctl->s_full);
+          ok = spin_bar_w(&ctl->st_full[0], 0, ctl);
+        }
+        if (ok) {
+          tc_fence_after();
           mma_ss_tiles<HD>(tmem + kTmemDP, sDO, sV);    // dP(0)
           umma_commit_w(&ctl->dp_full);
         }
@@ -608,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
           const int sn = (j + 1) % kStages;
           if (!(ok = spin_bar_w(&ctl->s_free, ph, ctl))) break;
           if (more) {
-            if (!(ok = spin_bar_w(&ctl->st_full[sn], (uint32_t)((j + 1) / kStages) & 1u, ctl)))
+            if (!(ok = spin_bar_w(&ctl->x_full[sn], (uint32_t)((j + 1) / kStages) & 1u, ctl)))
               break;
             tc_fence_after();
             mma_ss_tiles<HD>(tmem + kTmemS, sQ, sK + sn * L::kTileBytes);   // S(j+1)
@@ -622,6 +639,9 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
           if (!ok) break;
           umma_commit_w(&ctl->st_empty[st]);
           if (more) {
+            if (!(ok = spin_bar_w(&ctl->st_full[sn], (uint32_t)((j + 1) / kStages) & 1u, ctl)))
+              break;
+            tc_fence_after();
             mma_ss_tiles<HD>(tmem + kTmemDP, sDO, sV + sn * L::kTileBytes);  // dP(j+1)
             umma_commit_w(&ctl->dp_full);
           } else {
