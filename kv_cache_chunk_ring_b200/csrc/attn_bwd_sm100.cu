@@ -103,6 +103,44 @@ struct BwdSmem {
   static constexpr int kBytes = kCtl + (int)sizeof(BwdCtl) + 1024;
 };
 
+// dQ kernel: K_j streams through three slots, so the copy of K_{j+1} is not held
+// up until dQ_{j-1} has read K_{j-1}; V_j through two (freed after dP_j).  The
+// key-tile list is a ring the producer fills as it goes.  224 KB of tiles.
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kRing = 8;
+
+struct __align__(8) DqCtl {
+  uint64_t fixed_full;                         // Q_i, dO_i
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full, dp_full, s_free;
+  uint64_t ds_full[2];                         // per warpgroup (column half)
+  uint64_t acc_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int n_tiles;
+  int pad;
+  unsigned long long wait_ns;
+  uint16_t tiles[kRing];                       // key tile | class << 12, by j % kRing
+};
+
+// Offsets from the first 1024-byte aligned address of the dynamic shared memory;
+// the launch asks for at most the per-CTA limit, and the kernel checks the fit.
+template <int HD>
+struct DqSmem {
+  static constexpr int kTileBytes = BwdSmem<HD>::kTileBytes;
+  static constexpr int kQ = 0;
+  static constexpr int kDO = kQ + kTileBytes;
+  static constexpr int kK = kDO + kTileBytes;
+  static constexpr int kV = kK + kKStages * kTileBytes;
+  static constexpr int kCtl = kV + kVStages * kTileBytes;
+  static constexpr int kUsed = kCtl + (int)sizeof(DqCtl);
+  static constexpr int kBytes = kUsed + 1024 < 227 * 1024 ? kUsed + 1024 : 227 * 1024;
+};
+static_assert(DqSmem<128>::kUsed <= 227 * 1024, "dQ shared memory exceeds the per-CTA limit");
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -118,7 +156,8 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, BwdCtl* ctl) {
+template <class Ctl>
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Ctl* ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
@@ -133,7 +172,8 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, BwdCtl*
 }
 
 // wait_bar for the MMA-issuing warp: non-suspending polls.
-__device__ __forceinline__ bool spin_bar(uint64_t* bar, uint32_t parity, BwdCtl* ctl) {
+template <class Ctl>
+__device__ __forceinline__ bool spin_bar(uint64_t* bar, uint32_t parity, Ctl* ctl) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   uint32_t n = 0;
@@ -152,7 +192,8 @@ __device__ __forceinline__ bool spin_bar(uint64_t* bar, uint32_t parity, BwdCtl*
 
 // Time / abort check of a hand-written poll loop: true when the CTA is aborting or
 // the wait that began at t0 ran out (recording KVCR_ETIMEOUT and raising abort).
-__device__ __forceinline__ bool poll_expired(BwdCtl* ctl, uint64_t t0) {
+template <class Ctl>
+__device__ __forceinline__ bool poll_expired(Ctl* ctl, uint64_t t0) {
   if (*reinterpret_cast<volatile int*>(&ctl->abort)) return true;
   if (globaltimer() - t0 > ctl->wait_ns) {
     atomicExch(&g_bwd_status, (int)KVCR_ETIMEOUT);
@@ -165,7 +206,8 @@ __device__ __forceinline__ bool poll_expired(BwdCtl* ctl, uint64_t t0) {
 // spin_bar for the whole MMA warp: every lane polls (a completed phase stays
 // completed until the warp's own later products let the next one finish), and the
 // lanes agree on the outcome before the warp goes on, converged.
-__device__ __forceinline__ bool spin_bar_w(uint64_t* bar, uint32_t parity, BwdCtl* ctl) {
+template <class Ctl>
+__device__ __forceinline__ bool spin_bar_w(uint64_t* bar, uint32_t parity, Ctl* ctl) {
   const bool ok = spin_bar(bar, parity, ctl);
   return __all_sync(0xFFFFFFFFu, ok);
 }
@@ -205,11 +247,11 @@ __device__ __forceinline__ void load_tile(const CUtensorMap* m, uint8_t* dst, ui
     tma_load_3d(dst + b * BwdSmem<HD>::kBoxBytes, m, bar, b * 64, h, row0);
 }
 
-// List the tiles streamed past the CTA's own tile `t` (one warp): for the dK/dV
-// kernel (kByKey) the query tiles that may read key tile t, for the dQ kernel
-// the key tiles query tile t may read, each with its class.
+// Bounding range [u0, u1) of the tiles streamed past tile t: for the dK/dV kernel
+// (kByKey) the query tiles that may read key tile t, for the dQ kernel the key
+// tiles query tile t may read.
 template <bool kByKey>
-__device__ void build_list(const MobaBwdParams& p, int t, BwdCtl* ctl, int lane) {
+__device__ __forceinline__ void list_range(const MobaBwdParams& p, int t, int& u0, int& u1) {
   const MobaLay lay{p.s.n_chunks, p.s.chunk_tokens, p.s.n_bidir, p.s.L};
   const int r0 = t * kTile;
   const int r1 = min(r0 + kTile, p.s.L);
@@ -218,19 +260,65 @@ __device__ void build_list(const MobaBwdParams& p, int t, BwdCtl* ctl, int lane)
     moba_col_bounds(lay, r0, r1, lo, hi);
   else
     moba_row_bounds(lay, r0, r1, lo, hi);
-  const int u0 = lo / kTile, u1 = hi > lo ? (hi + kTile - 1) / kTile : u0;
+  u0 = lo / kTile;
+  u1 = hi > lo ? (hi + kTile - 1) / kTile : u0;
+}
+
+// Class of the pair (tile t, streamed tile u).
+template <bool kByKey>
+__device__ __forceinline__ int pair_class(const MobaBwdParams& p, int t, int u) {
+  const MobaLay lay{p.s.n_chunks, p.s.chunk_tokens, p.s.n_bidir, p.s.L};
+  return kByKey ? moba_classify(lay, u, t, kTile) : moba_classify(lay, t, u, kTile);
+}
+
+// Count (one warp) the non-empty tiles of that range and, when `tiles` is given,
+// list them in order, each with its class (u | class << 12).
+template <bool kByKey>
+__device__ int build_list(const MobaBwdParams& p, int t, uint16_t* tiles, int lane) {
+  int u0, u1;
+  list_range<kByKey>(p, t, u0, u1);
   int count = 0;
   for (int base = u0; base < u1; base += 32) {
     const int u = base + lane;
-    int c = kTileEmpty;
-    if (u < u1) c = kByKey ? moba_classify(lay, u, t, kTile) : moba_classify(lay, t, u, kTile);
+    const int c = u < u1 ? pair_class<kByKey>(p, t, u) : (int)kTileEmpty;
     const bool keep = c != kTileEmpty;
     const unsigned ball = __ballot_sync(0xFFFFFFFFu, keep);
-    if (keep) ctl->tiles[count + __popc(ball & ((1u << lane) - 1u))] = (uint16_t)(u | (c << 12));
+    if (keep && tiles) tiles[count + __popc(ball & ((1u << lane) - 1u))] = (uint16_t)(u | (c << 12));
     count += __popc(ball);
   }
-  if (lane == 0) ctl->n_tiles = count;
+  return count;
 }
+
+// The non-empty streamed tiles of [u0, u1) in order, found by the whole warp 32
+// candidates at a time (one ballot per block of 32, as build_list); every lane
+// gets the same (u, class) from next().
+template <bool kByKey>
+struct TileFeeder {
+  const MobaBwdParams& p;
+  int t, lane, base, u1, cls;
+  unsigned mask;
+  __device__ __forceinline__ TileFeeder(const MobaBwdParams& p_, int t_, int lane_)
+      : p(p_), t(t_), lane(lane_), cls(kTileEmpty), mask(0u) {
+    int u0;
+    list_range<kByKey>(p, t, u0, u1);
+    base = u0 - 32;
+  }
+  // false when the range is exhausted
+  __device__ __forceinline__ bool next(int& u, int& c) {
+    while (mask == 0u) {
+      base += 32;
+      if (base >= u1) return false;
+      const int v = base + lane;
+      cls = v < u1 ? pair_class<kByKey>(p, t, v) : (int)kTileEmpty;
+      mask = __ballot_sync(0xFFFFFFFFu, cls != kTileEmpty);
+    }
+    const int bit = __ffs(mask) - 1;
+    mask &= mask - 1u;
+    u = base + bit;
+    c = __shfl_sync(0xFFFFFFFFu, cls, bit);
+    return true;
+  }
+};
 
 // Shared prologue: barriers, TMEM, work list.  Returns the CTA's own tile.
 template <bool kByKey>
@@ -261,7 +349,10 @@ __device__ __forceinline__ void bwd_setup(const MobaBwdParams& p, BwdCtl* ctl, i
     tmem_alloc(&ctl->tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kWarpTma) build_list<kByKey>(p, tile, ctl, lane);
+  if (warp == kWarpTma) {
+    const int n = build_list<kByKey>(p, tile, ctl->tiles, lane);
+    if (lane == 0) ctl->n_tiles = n;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -582,68 +673,171 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
 }
 
 // ----------------------------------------------------------------------- dQ --
+// Prologue of the dQ kernel: barriers, TMEM, the count of streamed key tiles.
+__device__ __forceinline__ void dq_setup(const MobaBwdParams& p, DqCtl* ctl, int qt, int warp,
+                                         int lane) {
+  if (threadIdx.x == 0) {
+    mbar_init(&ctl->fixed_full, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&ctl->k_full[s], 1);
+      mbar_init(&ctl->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&ctl->v_full[s], 1);
+      mbar_init(&ctl->v_empty[s], 1);
+    }
+    mbar_init(&ctl->s_full, 1);
+    mbar_init(&ctl->dp_full, 1);
+    mbar_init(&ctl->s_free, 256);
+    for (int w = 0; w < 2; ++w) mbar_init(&ctl->ds_full[w], 128);
+    mbar_init(&ctl->acc_done, 1);
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    ctl->wait_ns =
+        p.wait_ns > 0 ? (unsigned long long)p.wait_ns : (unsigned long long)kWaitTimeoutNs;
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTma) {
+    const int n = build_list<false>(p, qt, nullptr, lane);
+    if (lane == 0) ctl->n_tiles = n;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+// TMA producer of the dQ kernel (warp 8; lane 0 issues the copies): Q_i and dO_i,
+// then, for each key tile query tile i may read in order, its ring entry, K_j into
+// slot j % 3 and V_j into slot j % 2.
+template <int HD>
+__device__ void dq_producer(const MobaBwdParams& p, DqCtl* ctl, uint8_t* smem, int h, int qt,
+                            int lane) {
+  using L = DqSmem<HD>;
+  const int n_tiles = ctl->n_tiles;
+  if (lane == 0) {
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_k);
+    prefetch_tmap(&p.tm_v);
+    prefetch_tmap(&p.tm_do);
+    mbar_arrive_expect_tx(&ctl->fixed_full, 2 * L::kTileBytes);
+    load_tile<HD>(&p.tm_q, smem + L::kQ, &ctl->fixed_full, h, qt * kTile);
+    load_tile<HD>(&p.tm_do, smem + L::kDO, &ctl->fixed_full, h, qt * kTile);
+  }
+  TileFeeder<false> feed(p, qt, lane);
+  int nk = 0, nv = 0;  // copies issued
+  bool ok = true;
+  for (int j = 0; j < n_tiles; ++j) {
+    int u, c;
+    if (!feed.next(u, c)) {  // unreachable: n_tiles counts the same classification
+      if (lane == 0) {
+        atomicExch(&g_bwd_status, (int)KVCR_ESTATE);
+        *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+      }
+      ok = false;
+      break;
+    }
+    const int ks = j % kKStages;
+    ok = __all_sync(0xFFFFFFFFu,
+                    wait_bar(&ctl->k_empty[ks], ((uint32_t)(j / kKStages) & 1u) ^ 1u, ctl));
+    if (!ok) break;
+    if (lane == 0) {
+      ctl->tiles[j % kRing] = (uint16_t)(u | (c << 12));
+      mbar_arrive_expect_tx(&ctl->k_full[ks], L::kTileBytes);
+      load_tile<HD>(&p.tm_k, smem + L::kK + ks * L::kTileBytes, &ctl->k_full[ks], h, u * kTile);
+    }
+    nk = j + 1;
+    const int vs = j % kVStages;
+    ok = __all_sync(0xFFFFFFFFu,
+                    wait_bar(&ctl->v_empty[vs], ((uint32_t)(j / kVStages) & 1u) ^ 1u, ctl));
+    if (!ok) break;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&ctl->v_full[vs], L::kTileBytes);
+      load_tile<HD>(&p.tm_v, smem + L::kV + vs * L::kTileBytes, &ctl->v_full[vs], h, u * kTile);
+    }
+    nv = j + 1;
+  }
+  if (!ok && lane == 0) {
+    // let every issued copy land before the CTA can exit
+    drain_wait(&ctl->fixed_full, 0);
+    for (int j = nk - kKStages < 0 ? 0 : nk - kKStages; j < nk; ++j)
+      drain_wait(&ctl->k_full[j % kKStages], (uint32_t)(j / kKStages) & 1u);
+    for (int j = nv - kVStages < 0 ? 0 : nv - kVStages; j < nv; ++j)
+      drain_wait(&ctl->v_full[j % kVStages], (uint32_t)(j / kVStages) & 1u);
+  }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_constant__ MobaBwdParams p) {
-  using L = BwdSmem<HD>;
+  using L = DqSmem<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  BwdCtl* ctl = reinterpret_cast<BwdCtl*>(smem + L::kCtl);
+  if ((int)(smem - smem_raw) + L::kUsed > L::kBytes) {  // uniform: before any barrier
+    if (threadIdx.x == 0) atomicExch(&g_bwd_status, (int)KVCR_EUNSUPPORTED);
+    return;
+  }
+  DqCtl* ctl = reinterpret_cast<DqCtl*>(smem + L::kCtl);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int h = blockIdx.x / p.s.n_units;             // head-major: co-resident CTAs
   const int qt = p.s.order[blockIdx.x - h * p.s.n_units];  // share one head in L2
   const int q0 = qt * kTile;
 
-  bwd_setup<false>(p, ctl, qt, warp, lane);
+  dq_setup(p, ctl, qt, warp, lane);
   const uint32_t tmem = ctl->tmem_base;
   const int n_tiles = ctl->n_tiles;
 
   if (warp >= 8) {
     setmaxnreg_dec<kRegsProducer>();
     if (warp == kWarpTma) {
-      if (lane == 0 && n_tiles > 0) bwd_producer<HD, false>(p, ctl, smem, h, qt);
+      if (n_tiles > 0) dq_producer<HD>(p, ctl, smem, h, qt, lane);
     } else if (warp == kWarpMma) {
       if (n_tiles > 0) {          // the whole warp: operands stay warp-uniform
-        const uint32_t sQ = smem_u32(smem + L::kA), sDO = smem_u32(smem + L::kB);
-        const uint32_t sK = smem_u32(smem + L::kX), sV = smem_u32(smem + L::kY);
-        bool ok = spin_bar_w(&ctl->fixed_full, 0, ctl) && spin_bar_w(&ctl->x_full[0], 0, ctl);
+        const uint32_t sQ = smem_u32(smem + L::kQ), sDO = smem_u32(smem + L::kDO);
+        const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+        bool ok = spin_bar_w(&ctl->fixed_full, 0, ctl) && spin_bar_w(&ctl->k_full[0], 0, ctl);
         if (ok) {
           tc_fence_after();
           mma_ss_tiles<HD>(tmem + kTmemS, sQ, sK);      // S(0)
           umma_commit_w(&ctl->s_full);
-          ok = spin_bar_w(&ctl->st_full[0], 0, ctl);
+          ok = spin_bar_w(&ctl->v_full[0], 0, ctl);
         }
         if (ok) {
           tc_fence_after();
           mma_ss_tiles<HD>(tmem + kTmemDP, sDO, sV);    // dP(0)
           umma_commit_w(&ctl->dp_full);
+          umma_commit_w(&ctl->v_empty[0]);              // last read of V_0
         }
         for (int j = 0; ok && j < n_tiles; ++j) {
-          const int st = j % kStages;
           const bool more = j + 1 < n_tiles;
           const uint32_t ph = (uint32_t)j & 1u;
-          const int sn = (j + 1) % kStages;
+          const int ks = j % kKStages, kn = (j + 1) % kKStages;
+          const int vn = (j + 1) % kVStages;
           if (!(ok = spin_bar_w(&ctl->s_free, ph, ctl))) break;
           if (more) {
-            if (!(ok = spin_bar_w(&ctl->x_full[sn], (uint32_t)((j + 1) / kStages) & 1u, ctl)))
+            if (!(ok = spin_bar_w(&ctl->k_full[kn], (uint32_t)((j + 1) / kKStages) & 1u, ctl)))
               break;
             tc_fence_after();
-            mma_ss_tiles<HD>(tmem + kTmemS, sQ, sK + sn * L::kTileBytes);   // S(j+1)
+            mma_ss_tiles<HD>(tmem + kTmemS, sQ, sK + kn * L::kTileBytes);   // S(j+1)
             umma_commit_w(&ctl->s_full);
           }
           for (int w = 0; ok && w < 2; ++w) {           // dQ += dS K_j
             if (!(ok = spin_bar_w(&ctl->ds_full[w], ph, ctl))) break;
             tc_fence_after();
-            mma_ts_half<HD>(tmem + kTmemAcc0, tmem + kTmemDP, sK + st * L::kTileBytes, w, j == 0);
+            mma_ts_half<HD>(tmem + kTmemAcc0, tmem + kTmemDP, sK + ks * L::kTileBytes, w, j == 0);
           }
           if (!ok) break;
-          umma_commit_w(&ctl->st_empty[st]);
+          umma_commit_w(&ctl->k_empty[ks]);             // last read of K_j
           if (more) {
-            if (!(ok = spin_bar_w(&ctl->st_full[sn], (uint32_t)((j + 1) / kStages) & 1u, ctl)))
+            if (!(ok = spin_bar_w(&ctl->v_full[vn], (uint32_t)((j + 1) / kVStages) & 1u, ctl)))
               break;
             tc_fence_after();
-            mma_ss_tiles<HD>(tmem + kTmemDP, sDO, sV + sn * L::kTileBytes);  // dP(j+1)
+            mma_ss_tiles<HD>(tmem + kTmemDP, sDO, sV + vn * L::kTileBytes);  // dP(j+1)
             umma_commit_w(&ctl->dp_full);
+            umma_commit_w(&ctl->v_empty[vn]);           // last read of V_{j+1}
           } else {
             umma_commit_w(&ctl->acc_done);
           }
@@ -675,14 +869,16 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
     bool ok = true;
 
     for (int j = 0; j < n_tiles; ++j) {
-      const uint32_t e = ctl->tiles[j];
-      const int kt = (int)(e & 0xFFFu);
-      const int cls = (int)((e >> 12) & 3u);
-      ok = wait_bar(&ctl->s_full, (uint32_t)j & 1u, ctl);
+      // K_j's copy (and with it this ring entry) has landed, and S(j) is in TMEM
+      ok = wait_bar(&ctl->k_full[j % kKStages], (uint32_t)(j / kKStages) & 1u, ctl) &&
+           wait_bar(&ctl->s_full, (uint32_t)j & 1u, ctl);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         ok = false;
         break;
       }
+      const uint32_t e = ctl->tiles[j % kRing];
+      const int kt = (int)(e & 0xFFFu);
+      const int cls = (int)((e >> 12) & 3u);
       tc_fence_after();
       uint32_t s[64];
       tmem_ld_32x32b_x32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
@@ -849,11 +1045,11 @@ cudaError_t launch_dq(const MobaBwdParams& p, cudaStream_t s) {
     return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<HD>::kBytes);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DqSmem<HD>::kBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  kern<<<(unsigned)(p.s.n_units * p.H), kThreads, BwdSmem<HD>::kBytes, s>>>(p);
+  kern<<<(unsigned)(p.s.n_units * p.H), kThreads, DqSmem<HD>::kBytes, s>>>(p);
   return cudaGetLastError();
 }
 
