@@ -16,7 +16,8 @@
 //          their probabilities are exactly 0.
 //   dK/dV  one CTA per (head, 128-key tile), head-major and heaviest tiles first
 //          within a head; K_j, V_j stay in shared memory and
-//          the query tiles that may read them stream through a 2-stage ring:
+//          the query tiles that may read them stream through a 2-stage ring
+//          (Q_i copied first, under a barrier of its own):
 //            S^T  = K_j Q_i^T            (SS)       TMEM cols   0-127
 //            dP^T = V_j dO_i^T           (SS)       TMEM cols 128-255
 //            dV  += P^T dO_i             (TS: P^T in TMEM, dO_i MN-major)  256-383
@@ -31,7 +32,8 @@
 //          of dV_i when it can, and overlaps tile i's exponentials; dP^T(i+1)
 //          follows dK_i (MMAs of one thread run in issue order).
 //   dQ     one CTA per (head, 128-query tile), the key tiles it may read
-//          streaming through the ring:
+//          streaming K_j through three slots and V_j through two (the producer
+//          warp finds the tiles 32 per ballot and hands them on in a ring):
 //            S  = Q K_j^T (SS, cols 0-127)   dP = dO V_j^T (SS, cols 128-255)
 //            dQ += dS K_j (TS: dS in TMEM, K_j MN-major; cols 256-383)
 //          Thread r owns query r; LSE and D are per row (registers).
