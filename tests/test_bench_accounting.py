@@ -42,3 +42,45 @@ def test_append_bytes():
     spec = wl.VIDEO_832x464
     # K and V of 4 frames of 1508 tokens x 12 heads x 128, bf16, each read once and written once
     assert bench.append_bytes(spec) == 2 * 2 * 4 * 1508 * 12 * 128 * 2
+
+
+def test_clock_samples_outside_the_timed_window_are_dropped(tmp_path):
+    """The clock summary keeps only nvidia-smi samples stamped inside the timed region:
+    idle samples before it (the sampler starts early) must not pull the median down,
+    and a throttle reason seen only outside it is not reported."""
+    import time
+
+    import bench
+
+    def stamp(t):
+        return time.strftime("%Y/%m/%d %H:%M:%S", time.localtime(t)) + ".%03d" % int((t % 1) * 1000)
+
+    t0 = time.mktime(time.strptime("2026/12/03 10:00:00", "%Y/%m/%d %H:%M:%S"))
+    rows = [  # (time, sm clock, sw_power_cap)
+        (t0 - 0.40, 345, "Not Active"),   # idle, before the window
+        (t0 - 0.10, 1965, "Active"),      # before the window, power cap
+        (t0 + 0.05, 1965, "Not Active"),
+        (t0 + 0.10, 1950, "Not Active"),
+        (t0 + 0.15, 1935, "Not Active"),
+        (t0 + 0.60, 300, "Active"),       # after the window
+    ]
+    path = tmp_path / "clocks.csv"
+    with open(path, "w") as f:
+        for t, clk, cap in rows:
+            f.write(f"{stamp(t)}, 0, {clk}, 1965, 700.00, 0x0, Not Active, Not Active, "
+                    f"Not Active, {cap}\n")
+
+    class _Proc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    s = bench.ClockSampler(0)
+    s.path = str(path)
+    s.proc = _Proc()
+    s.f = open(path, "a")
+    s.window(t0, t0 + 0.2)
+    got = s.stop()
+    assert got == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 3}
