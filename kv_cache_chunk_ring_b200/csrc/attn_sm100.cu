@@ -66,12 +66,12 @@ constexpr float kRescaleLog2 = 8.0f;
 // P of a tile is released to the MMA in this many parts of 128 / kPParts keys.
 constexpr int kPParts = 2;
 // Of the 16 key pairs in each 32-key group, pairs [0, kExpSfuPairs) take exp2 on
-// the SFU and the rest on the FMA pipe.  With bf16 QK^T all go to the SFU; with
-// the e4m3 QK^T (half the S product time) moving 2 of 16 pairs to the FMA pipe
-// measured 4-5 % faster (0.78 against 0.81-0.82 ms per 832x464 call), while the
-// same split slowed the bf16 kernel by about 1 %.
+// the SFU and the rest on the FMA pipe.  With bf16 QK^T all go to the SFU (1 or 2
+// of 16 on the FMA pipe measured the same or ~1 % slower); with the e4m3 QK^T
+// (half the S product time) 4 of 16 on the FMA pipe measured fastest per 832x464
+// call: 0.768 ms against 0.780 with 2 of 16, 0.786 with 6 of 16, 0.81-0.82 with none.
 constexpr int kExpSfuPairs = 16;
-constexpr int kExpSfuPairsE4m3 = 14;
+constexpr int kExpSfuPairsE4m3 = 12;
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S_t / P_t at t * 128, O_t at 256 + t * 128.
 constexpr uint32_t kTmemS = 0;
