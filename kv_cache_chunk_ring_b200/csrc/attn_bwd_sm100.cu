@@ -77,7 +77,7 @@ constexpr int kWsBytes = kTile * 8;  // (lse, D) of one 128-row tile
 
 struct __align__(8) BwdCtl {
   uint64_t fixed_full;                         // the CTA's own two tiles
-  uint64_t x_full[kStages];                    // stage: first streamed tile (Q_i or K_j)
+  uint64_t x_full[kStages];                    // stage: Q_i
   uint64_t st_full[kStages], st_empty[kStages];  // the rest of the stage; the whole stage
   uint64_t s_full, dp_full, s_free;
   uint64_t p_full[2], ds_full[2];              // per warpgroup (column half)
@@ -96,10 +96,10 @@ struct BwdSmem {
   static constexpr int kBoxes = HD / 64;
   static constexpr int kBoxBytes = 128 * 128;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kA = 0;                              // K_j (dK/dV) or Q_i (dQ)
-  static constexpr int kB = kA + kTileBytes;                // V_j or dO_i
-  static constexpr int kX = kB + kTileBytes;                // stages: Q_i or K_j
-  static constexpr int kY = kX + kStages * kTileBytes;      // stages: dO_i or V_j
+  static constexpr int kA = 0;                              // K_j   (dK/dV kernel)
+  static constexpr int kB = kA + kTileBytes;                // V_j
+  static constexpr int kX = kB + kTileBytes;                // stages: Q_i
+  static constexpr int kY = kX + kStages * kTileBytes;      // stages: dO_i
   static constexpr int kW = kY + kStages * kTileBytes;      // stages: (lse, D) of Q_i
   static constexpr int kCtl = kW + kStages * kWsBytes;
   static constexpr int kBytes = kCtl + (int)sizeof(BwdCtl) + 1024;
@@ -322,10 +322,9 @@ struct TileFeeder {
   }
 };
 
-// Shared prologue: barriers, TMEM, work list.  Returns the CTA's own tile.
-template <bool kByKey>
-__device__ __forceinline__ void bwd_setup(const MobaBwdParams& p, BwdCtl* ctl, int tile,
-                                          int warp, int lane) {
+// Prologue of the dK/dV kernel: barriers, TMEM, the list of streamed query tiles.
+__device__ __forceinline__ void dkdv_setup(const MobaBwdParams& p, BwdCtl* ctl, int tile,
+                                           int warp, int lane) {
   if (threadIdx.x == 0) {
     mbar_init(&ctl->fixed_full, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -352,7 +351,7 @@ __device__ __forceinline__ void bwd_setup(const MobaBwdParams& p, BwdCtl* ctl, i
     tmem_relinquish();
   }
   if (warp == kWarpTma) {
-    const int n = build_list<kByKey>(p, tile, ctl->tiles, lane);
+    const int n = build_list<true>(p, tile, ctl->tiles, lane);
     if (lane == 0) ctl->n_tiles = n;
   }
   tc_fence_before();
@@ -360,27 +359,23 @@ __device__ __forceinline__ void bwd_setup(const MobaBwdParams& p, BwdCtl* ctl, i
   tc_fence_after();
 }
 
-// TMA producer (one thread): the CTA's two fixed tiles, then per streamed tile
-// its two tiles (and, for the dK/dV kernel, the 1 KB of (lse, D) of its rows).
-template <int HD, bool kByKey>
-__device__ void bwd_producer(const MobaBwdParams& p, BwdCtl* ctl, uint8_t* smem, int h,
-                             int tile) {
+// TMA producer of the dK/dV kernel (one thread): K_j and V_j, then per streamed
+// query tile its Q_i, dO_i and the 1 KB of (lse, D) of its rows.
+template <int HD>
+__device__ void dkdv_producer(const MobaBwdParams& p, BwdCtl* ctl, uint8_t* smem, int h,
+                              int tile) {
   using L = BwdSmem<HD>;
   const int n_tiles = ctl->n_tiles;
   prefetch_tmap(&p.tm_q);
   prefetch_tmap(&p.tm_k);
   prefetch_tmap(&p.tm_v);
   prefetch_tmap(&p.tm_do);
-  const CUtensorMap* fa = kByKey ? &p.tm_k : &p.tm_q;
-  const CUtensorMap* fb = kByKey ? &p.tm_v : &p.tm_do;
-  const CUtensorMap* sx = kByKey ? &p.tm_q : &p.tm_k;
-  const CUtensorMap* sy = kByKey ? &p.tm_do : &p.tm_v;
   mbar_arrive_expect_tx(&ctl->fixed_full, 2 * L::kTileBytes);
-  load_tile<HD>(fa, smem + L::kA, &ctl->fixed_full, h, tile * kTile);
-  load_tile<HD>(fb, smem + L::kB, &ctl->fixed_full, h, tile * kTile);
-  // the first streamed tile (Q_i, K_j) is copied first and has a barrier of its
-  // own: the next S-type product needs only it, and starts before the rest lands
-  constexpr uint32_t kRestBytes = L::kTileBytes + (kByKey ? kWsBytes : 0);
+  load_tile<HD>(&p.tm_k, smem + L::kA, &ctl->fixed_full, h, tile * kTile);
+  load_tile<HD>(&p.tm_v, smem + L::kB, &ctl->fixed_full, h, tile * kTile);
+  // Q_i is copied first and has a barrier of its own: the next S^T needs only it,
+  // and starts before dO_i and (lse, D) land
+  constexpr uint32_t kRestBytes = L::kTileBytes + kWsBytes;
   int issued = 0;
   bool ok = true;
   for (int i = 0; i < n_tiles; ++i) {
@@ -389,12 +384,11 @@ __device__ void bwd_producer(const MobaBwdParams& p, BwdCtl* ctl, uint8_t* smem,
     const int u = (int)(ctl->tiles[i] & 0xFFFu);
     if (!(ok = wait_bar(&ctl->st_empty[st], ph ^ 1u, ctl))) break;
     mbar_arrive_expect_tx(&ctl->x_full[st], L::kTileBytes);
-    load_tile<HD>(sx, smem + L::kX + st * L::kTileBytes, &ctl->x_full[st], h, u * kTile);
+    load_tile<HD>(&p.tm_q, smem + L::kX + st * L::kTileBytes, &ctl->x_full[st], h, u * kTile);
     mbar_arrive_expect_tx(&ctl->st_full[st], kRestBytes);
-    load_tile<HD>(sy, smem + L::kY + st * L::kTileBytes, &ctl->st_full[st], h, u * kTile);
-    if (kByKey)
-      bulk_load(smem + L::kW + st * kWsBytes, p.ws + ((size_t)h * p.s.n_units + u) * 2 * kTile,
-                kWsBytes, &ctl->st_full[st]);
+    load_tile<HD>(&p.tm_do, smem + L::kY + st * L::kTileBytes, &ctl->st_full[st], h, u * kTile);
+    bulk_load(smem + L::kW + st * kWsBytes, p.ws + ((size_t)h * p.s.n_units + u) * 2 * kTile,
+              kWsBytes, &ctl->st_full[st]);
     issued = i + 1;
   }
   if (!ok) {
@@ -446,14 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
   const int kt = p.s.order[blockIdx.x - h * p.s.n_units];  // share one head in L2
   const int k0 = kt * kTile;
 
-  bwd_setup<true>(p, ctl, kt, warp, lane);
+  dkdv_setup(p, ctl, kt, warp, lane);
   const uint32_t tmem = ctl->tmem_base;
   const int n_tiles = ctl->n_tiles;
 
   if (warp >= 8) {
     setmaxnreg_dec<kRegsProducer>();
     if (warp == kWarpTma) {
-      if (lane == 0 && n_tiles > 0) bwd_producer<HD, true>(p, ctl, smem, h, kt);
+      if (lane == 0 && n_tiles > 0) dkdv_producer<HD>(p, ctl, smem, h, kt);
     } else if (warp == kWarpMma) {
       if (n_tiles > 0) {          // the whole warp: operands stay warp-uniform
         const uint32_t sK = smem_u32(smem + L::kA), sV = smem_u32(smem + L::kB);
