@@ -39,7 +39,11 @@
  *  - A failure inside a kernel (a bounded wait that ran out) happens after the
  *    launching call has returned KVCR_OK: poll kvcr_check_status() after the
  *    stream's work to learn of it; until then the outputs of that work are
- *    not to be trusted.
+ *    not to be trusted.  Besides KVCR_ETIMEOUT, the MoBA backward's dQ kernel
+ *    records two self-checks there, neither expected on sm_100: KVCR_EUNSUPPORTED
+ *    when its shared-memory layout does not fit the block's dynamic shared
+ *    memory after alignment, KVCR_ESTATE when its enumeration of key tiles
+ *    disagrees with its own count; the kernel then stops without touching dQ.
  */
 #ifndef KVCR_H
 #define KVCR_H
