@@ -11,9 +11,10 @@
 // in fp32 on the tensor cores (bf16 operands), written back as bf16.
 //
 // Three launches, no atomics (the result does not depend on scheduling):
-//   prep   per head and 128-row tile: LSE_i * log2 e of its rows, then D_i of
-//          them (ws[h][t][0][r], ws[h][t][1][r]); rows past L get (+inf, 0), so
-//          their probabilities are exactly 0.
+//   prep   per head and 128-row tile: LSE_i * log2 e of its rows, then -D_i of
+//          them (ws[h][t][0][r], ws[h][t][1][r]; negated so that dP - D is one
+//          packed add); rows past L get (+inf, 0), so their probabilities are
+//          exactly 0.
 //   dK/dV  one CTA per (head, 128-key tile), head-major and heaviest tiles first
 //          within a head; K_j, V_j stay in shared memory and
 //          the query tiles that may read them stream through a 2-stage ring
@@ -46,6 +47,8 @@
 // drains its copies and MMAs before freeing TMEM.
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <type_traits>
 
 #include "attn_bwd.h"
 #include "moba_layout.h"
@@ -239,6 +242,17 @@ __device__ __forceinline__ float ex2_sfu(float x) {
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Packed two-lane fp32 product (sm_100): one instruction for two values.
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
 template <int HD>
@@ -559,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&ctl->s_free);                    // S^T columns may take S^T(i+1)
-      // lse * log2 e (l4) and D (d4) of columns 4m .. 4m + 3 of this warpgroup
+      // lse * log2 e (l4) and -D (d4) of columns 4m .. 4m + 3 of this warpgroup
       const float4* l4 = reinterpret_cast<const float4*>(smem + L::kW + st * kWsBytes) + wg * 16;
       const float4* d4 = l4 + kTile / 4;
       uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
@@ -572,18 +586,26 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
       }
       float pr[64];
       const float2 sl2x2 = make_float2(sl2, sl2);
+      // full tiles (most of them) skip the per-element mask
+      auto exps = [&](auto masked_c) {
+        constexpr bool kMasked = decltype(masked_c)::value;
 #pragma unroll
-      for (int n = 0; n < 64; n += 2) {
-        const float4 lv = l4[n >> 2];
-        const float2 x = ffma2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])),
-                               sl2x2, (n & 2) ? make_float2(-lv.z, -lv.w)
-                                              : make_float2(-lv.x, -lv.y));
-        float p0 = ex2_sfu(x.x), p1 = ex2_sfu(x.y);
-        if (!((keep[n >> 5] >> (n & 31)) & 1u)) p0 = 0.f;
-        if (!((keep[n >> 5] >> ((n + 1) & 31)) & 1u)) p1 = 0.f;
-        pr[n] = p0;
-        pr[n + 1] = p1;
-      }
+        for (int n = 0; n < 64; n += 2) {
+          const float4 lv = l4[n >> 2];
+          const float2 x = ffma2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])),
+                                 sl2x2, (n & 2) ? make_float2(-lv.z, -lv.w)
+                                                : make_float2(-lv.x, -lv.y));
+          float p0 = ex2_sfu(x.x), p1 = ex2_sfu(x.y);
+          if (kMasked) {
+            if (!((keep[n >> 5] >> (n & 31)) & 1u)) p0 = 0.f;
+            if (!((keep[n >> 5] >> ((n + 1) & 31)) & 1u)) p1 = 0.f;
+          }
+          pr[n] = p0;
+          pr[n + 1] = p1;
+        }
+      };
+      if (cls == kTileFull) exps(std::false_type{});
+      else exps(std::true_type{});
 
       ok = wait_bar(&ctl->dp_full, (uint32_t)i & 1u, ctl);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
@@ -613,10 +635,11 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const int n = 32 * c + 2 * q;
-          const float4 dv = d4[n >> 2];
-          const float d0 = pr[n] * (__uint_as_float(s[n]) - ((q & 1) ? dv.z : dv.x));
-          const float d1 = pr[n + 1] * (__uint_as_float(s[n + 1]) - ((q & 1) ? dv.w : dv.y));
-          packed[q] = pack_bf16(d0, d1);
+          const float4 nd = d4[n >> 2];                 // -D of the columns
+          const float2 t = fadd2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])),
+                                 (q & 1) ? make_float2(nd.z, nd.w) : make_float2(nd.x, nd.y));
+          const float2 d = fmul2(make_float2(pr[n], pr[n + 1]), t);
+          packed[q] = pack_bf16(d.x, d.y);
         }
         tmem_st_32x32b_x16(dp_addr + 32 + c * 16, packed);
       }
@@ -854,7 +877,8 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
     const float sl2 = p.scale_log2;
     const MobaLay lay{p.s.n_chunks, p.s.chunk_tokens, p.s.n_bidir, p.s.L};
     const float* wt = p.ws + ((size_t)h * p.s.n_units + qt) * 2 * kTile;
-    const float2 wrow = make_float2(wt[r], wt[kTile + r]);   // (lse * log2 e, D) of row q0 + r
+    const float2 wrow = make_float2(wt[r], wt[kTile + r]);   // (lse * log2 e, -D) of row q0 + r
+    const float2 neg_d = make_float2(wrow.y, wrow.y);
     const float2 sl2x2 = make_float2(sl2, sl2);
     const float2 neg_lse = make_float2(-wrow.x, -wrow.x);
     int a[2] = {0, 0}, b[2] = {0, 0};
@@ -892,16 +916,24 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
           keep[c] &= bit_range(a[0] - base, b[0] - base) | bit_range(a[1] - base, b[1] - base);
       }
       float pr[64];
+      // full tiles inside the sequence (most of them) skip the per-element mask
+      auto exps = [&](auto masked_c) {
+        constexpr bool kMasked = decltype(masked_c)::value;
 #pragma unroll
-      for (int n = 0; n < 64; n += 2) {
-        const float2 x =
-            ffma2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])), sl2x2, neg_lse);
-        float p0 = ex2_sfu(x.x), p1 = ex2_sfu(x.y);
-        if (!((keep[n >> 5] >> (n & 31)) & 1u)) p0 = 0.f;
-        if (!((keep[n >> 5] >> ((n + 1) & 31)) & 1u)) p1 = 0.f;
-        pr[n] = p0;
-        pr[n + 1] = p1;
-      }
+        for (int n = 0; n < 64; n += 2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])),
+                                 sl2x2, neg_lse);
+          float p0 = ex2_sfu(x.x), p1 = ex2_sfu(x.y);
+          if (kMasked) {
+            if (!((keep[n >> 5] >> (n & 31)) & 1u)) p0 = 0.f;
+            if (!((keep[n >> 5] >> ((n + 1) & 31)) & 1u)) p1 = 0.f;
+          }
+          pr[n] = p0;
+          pr[n + 1] = p1;
+        }
+      };
+      if (cls == kTileFull && (kt + 1) * kTile <= p.s.L) exps(std::false_type{});
+      else exps(std::true_type{});
 
       ok = wait_bar(&ctl->dp_full, (uint32_t)j & 1u, ctl);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
@@ -918,8 +950,10 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const int n = 32 * c + 2 * q;
-          packed[q] = pack_bf16(pr[n] * (__uint_as_float(s[n]) - wrow.y),
-                                pr[n + 1] * (__uint_as_float(s[n + 1]) - wrow.y));
+          const float2 t = fadd2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])),
+                                 neg_d);
+          const float2 d = fmul2(make_float2(pr[n], pr[n + 1]), t);
+          packed[q] = pack_bf16(d.x, d.y);
         }
         tmem_st_32x32b_x16(dp_addr + c * 16, packed);
       }
@@ -1009,7 +1043,7 @@ __global__ void __launch_bounds__(256) moba_bwd_prep_kernel(const MobaBwdPrepPar
     }
     float* wt = p.ws + ((size_t)h * (p.Lpad / kTile) + row / kTile) * 2 * kTile;
     wt[row % kTile] = lse2;
-    wt[kTile + row % kTile] = live ? acc : 0.f;
+    wt[kTile + row % kTile] = live ? -acc : 0.f;
   }
 }
 
