@@ -11,10 +11,10 @@
 // in fp32 on the tensor cores (bf16 operands), written back as bf16.
 //
 // Three launches, no atomics (the result does not depend on scheduling):
-//   prep   per head and 128-row tile: LSE_i * log2 e of its rows, then -D_i of
-//          them (ws[h][t][0][r], ws[h][t][1][r]; negated so that dP - D is one
-//          packed add); rows past L get (+inf, 0), so their probabilities are
-//          exactly 0.
+//   prep   per head and 128-row tile: -LSE_i * log2 e of its rows, then -D_i of
+//          them (ws[h][t][0][r], ws[h][t][1][r]; negated so that they enter the
+//          packed fma and add as they are); rows past L get (-inf, 0), so their
+//          probabilities are exactly 0.
 //   dK/dV  one CTA per (head, 128-key tile), head-major and heaviest tiles first
 //          within a head; K_j, V_j stay in shared memory and
 //          the query tiles that may read them stream through a 2-stage ring
@@ -573,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&ctl->s_free);                    // S^T columns may take S^T(i+1)
-      // lse * log2 e (l4) and -D (d4) of columns 4m .. 4m + 3 of this warpgroup
+      // -lse * log2 e (l4) and -D (d4) of columns 4m .. 4m + 3 of this warpgroup
       const float4* l4 = reinterpret_cast<const float4*>(smem + L::kW + st * kWsBytes) + wg * 16;
       const float4* d4 = l4 + kTile / 4;
       uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
@@ -593,8 +593,8 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dkdv_kernel(const __grid_con
         for (int n = 0; n < 64; n += 2) {
           const float4 lv = l4[n >> 2];
           const float2 x = ffma2(make_float2(__uint_as_float(s[n]), __uint_as_float(s[n + 1])),
-                                 sl2x2, (n & 2) ? make_float2(-lv.z, -lv.w)
-                                                : make_float2(-lv.x, -lv.y));
+                                 sl2x2, (n & 2) ? make_float2(lv.z, lv.w)
+                                                : make_float2(lv.x, lv.y));
           float p0 = ex2_sfu(x.x), p1 = ex2_sfu(x.y);
           if (kMasked) {
             if (!((keep[n >> 5] >> (n & 31)) & 1u)) p0 = 0.f;
@@ -877,10 +877,10 @@ __global__ void __launch_bounds__(kThreads, 1) moba_dq_kernel(const __grid_const
     const float sl2 = p.scale_log2;
     const MobaLay lay{p.s.n_chunks, p.s.chunk_tokens, p.s.n_bidir, p.s.L};
     const float* wt = p.ws + ((size_t)h * p.s.n_units + qt) * 2 * kTile;
-    const float2 wrow = make_float2(wt[r], wt[kTile + r]);   // (lse * log2 e, -D) of row q0 + r
+    const float2 wrow = make_float2(wt[r], wt[kTile + r]);   // (-lse * log2 e, -D) of row q0 + r
     const float2 neg_d = make_float2(wrow.y, wrow.y);
     const float2 sl2x2 = make_float2(sl2, sl2);
-    const float2 neg_lse = make_float2(-wrow.x, -wrow.x);
+    const float2 neg_lse = make_float2(wrow.x, wrow.x);
     int a[2] = {0, 0}, b[2] = {0, 0};
     {
       const int row = min(q0 + r, p.s.L - 1);
@@ -1042,7 +1042,7 @@ __global__ void __launch_bounds__(256) moba_bwd_prep_kernel(const MobaBwdPrepPar
       if (v != -INFINITY) lse2 = v * 1.4426950408889634f;
     }
     float* wt = p.ws + ((size_t)h * (p.Lpad / kTile) + row / kTile) * 2 * kTile;
-    wt[row % kTile] = lse2;
+    wt[row % kTile] = -lse2;                        // stored negated, as -D below
     wt[kTile + row % kTile] = live ? -acc : 0.f;
   }
 }
